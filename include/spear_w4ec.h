@@ -1,0 +1,147 @@
+/*
+ * spear_w4ec.h -- C ABI of the W4 + per-token-gated low-rank Error
+ * Compensator (EC) linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (SPEAR, "A System for Post-Quantization Error-Adaptive Recovery
+ * Enabling Efficient Low-Bit LLM Serving", Abstract): weights quantised to
+ * 4 bits per output channel, and a lightweight Error Compensator whose
+ * strength a per-token gate sets, with the correction fused into the low-bit
+ * GEMM and an adaptive choice between fused and unfused kernels.  The pages
+ * give no equations; this library computes
+ *
+ *   y[t,n] = sum_k x[t,k] * s[n]*(q[n,k] - z[n])  +  g_t * sum_j u[t,j] * B[j,n]
+ *   u[t,j] = sum_k x[t,k] * A[k,j]
+ *   g_t    = 1 / (1 + exp(-(sum_k x[t,k] * w_g[k] + b_g)))
+ *
+ * with q in {0..15} packed eight per uint32 (code of k = 8j+i in bits
+ * [4i, 4i+3] of word j of row n), s[n] = fp32(max_k |W[n,k]|) / 7,
+ * q = clamp(round_half_even(fp32(W/s)), -8, 7) + 8 and z[n] = 8.
+ *
+ * Conventions for every call:
+ *  - All matrices are row-major and dense (leading dimension = row length).
+ *  - bf16 means IEEE bfloat16 bit patterns (uint16); "dev" pointers are CUDA
+ *    device pointers on the handle's device, "host" pointers are host memory.
+ *  - `stream` is a cudaStream_t passed as an opaque pointer (NULL = the
+ *    legacy default stream).  Device work is enqueued on it; calls return
+ *    before it completes unless stated otherwise.
+ *  - Every call returns a spear_status; nothing throws across the ABI.
+ *    Argument errors are reported synchronously and leave all state
+ *    unchanged.  Errors raised by kernels while they run (non-finite
+ *    weights, a device-side wait that ran out of time) are sticky in a
+ *    device status word that spear_w4ec_sync_status() returns and clears.
+ *  - The caller owns every buffer it passes; the library keeps no pointer
+ *    to a caller buffer after the call's stream work completes.
+ *  - A handle may be used from one host thread at a time.  Its workspace is
+ *    shared by its forward calls, so forward calls on one handle must be
+ *    ordered (issue them on one stream, or synchronise between streams);
+ *    calls that overlap on the GPU race on the workspace.
+ */
+#ifndef SPEAR_W4EC_H
+#define SPEAR_W4EC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct spear_w4ec spear_w4ec; /* opaque, owned by the library */
+
+typedef enum spear_status {
+    SPEAR_OK = 0,
+    SPEAR_ERR_INVALID = -1,     /* bad argument: shape, NULL, alignment, M > max_M */
+    SPEAR_ERR_UNSUPPORTED = -2, /* valid arguments, but no kernel for this case */
+    SPEAR_ERR_NOMEM = -3,       /* a device or host allocation failed */
+    SPEAR_ERR_CUDA = -4,        /* a CUDA runtime call or kernel launch failed */
+    SPEAR_ERR_TIMEOUT = -5,     /* a device-side wait gave up (sticky) */
+    SPEAR_ERR_DEVICE = -6,      /* a kernel flagged bad data, e.g. non-finite W (sticky) */
+    SPEAR_ERR_STATE = -7        /* call out of order, e.g. forward before pack */
+} spear_status;
+
+/* Flags of spear_w4ec_forward.  Path flags force one kernel family instead of
+ * the dispatch table's choice and return SPEAR_ERR_UNSUPPORTED if it cannot
+ * run the shape. */
+enum {
+    SPEAR_EC_OFF = 1u,        /* drop the EC: the plain W4 GEMM, y = x.W^T */
+    SPEAR_FORCE_FUSED = 2u,   /* EC applied inside the GEMM's epilogue / accumulator */
+    SPEAR_FORCE_SPLIT = 4u,   /* EC applied by a separate kernel after the GEMM */
+    SPEAR_FORCE_DECODE = 8u,  /* CUDA-core-fed tensor-core split-K kernel (small M) */
+    SPEAR_FORCE_TC = 16u      /* tcgen05 / TMEM tile kernel (larger M) */
+};
+
+typedef struct spear_w4ec_opts {
+    int64_t max_M;   /* largest M forward will be called with (workspace size); <= 0: 4096 */
+    int32_t device;  /* CUDA device ordinal; < 0: the current device */
+} spear_w4ec_opts;
+
+/* Create a layer of K input features, N output features and EC rank r.
+ * K and N must be positive multiples of 8; 0 <= r <= 128 (r = 0: no EC).
+ * Allocates the packed weights and the workspace on the device (about
+ * N*K/2 bytes of codes plus small buffers); no data is packed yet.
+ * opts may be NULL.  On success *out receives the handle. */
+int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r,
+                      const spear_w4ec_opts *opts);
+
+/* Quantise and pack the layer (SPEAR, Abstract: per-channel 4-bit weights).
+ *   W    dev bf16 [N][K]  full-precision weights, 16-byte aligned, finite
+ *   A    dev bf16 [K][r]  EC down-projection (ignored if r == 0; may be NULL)
+ *   B    dev bf16 [r][N]  EC up-projection   (ignored if r == 0; may be NULL)
+ *   w_g  dev bf16 [K]     gate weights       (ignored if r == 0; may be NULL)
+ *   b_g                   gate bias
+ * The codes and scales are bit-identical to the definition above.  The inputs
+ * may be freed once the stream work of this call has completed.  A
+ * non-finite W is reported as SPEAR_ERR_DEVICE by spear_w4ec_sync_status. */
+int spear_w4ec_pack(spear_w4ec *h, const void *W, const void *A, const void *B,
+                    const void *w_g, float b_g, void *stream);
+
+/* y = x.W^T + g.(x.A).B for M tokens.
+ *   x  dev bf16 [M][K], 16-byte aligned;  y  dev bf16 [M][N], 16-byte aligned.
+ * 0 <= M <= max_M (M = 0 is a no-op).  flags: SPEAR_* above (0 = dispatch).
+ * The result is rounded once to bf16 (round to nearest even) from an fp32
+ * accumulation.  Kernels of one call are ordered on `stream`. */
+int spear_w4ec_forward(const spear_w4ec *h, const void *x, void *y, int64_t M,
+                       uint32_t flags, void *stream);
+
+/* The same as spear_w4ec_forward, with x and y in HOST memory: copies x to a
+ * device staging buffer, runs the forward and copies y back, all on `stream`,
+ * then synchronises the stream.  Pinned host memory gives the fastest copies.
+ * The staging buffers are allocated on the first call (max_M rows). */
+int spear_w4ec_forward_host(spear_w4ec *h, const void *x_host, void *y_host, int64_t M,
+                            uint32_t flags, void *stream);
+
+/* Free everything the handle owns (synchronises the device first). NULL is a no-op. */
+int spear_w4ec_destroy(spear_w4ec *h);
+
+/* Copy the packed layer out, in the exported layout:
+ *   codes dev uint32 [N][K/8], s dev float [N], z dev uint8 [N].
+ * Any of the three may be NULL to skip it. */
+int spear_w4ec_get_packed(const spear_w4ec *h, void *codes, float *s, uint8_t *z, void *stream);
+
+/* Per-token gate g_t for M tokens of x (dev bf16 [M][K]) into g (dev float [M]).
+ * Uses the same kernel as the forward pass's gate. Requires r > 0. */
+int spear_w4ec_get_gate(const spear_w4ec *h, const void *x, float *g, int64_t M, void *stream);
+
+/* Synchronise `stream`, then return and clear the sticky device status
+ * (SPEAR_OK, SPEAR_ERR_TIMEOUT or SPEAR_ERR_DEVICE). */
+int spear_w4ec_sync_status(spear_w4ec *h, void *stream);
+
+/* Adaptive kernel-fusion dispatch (SPEAR, Abstract): time every legal
+ * {kernel family} x {fused, split} choice for M tokens on the caller's x and
+ * y buffers (dev, shapes as in forward; y is overwritten), record the fastest
+ * in the handle's table for M's bucket (1,2,4,...,128, 256+) and return its
+ * flags in *choice (may be NULL).  Synchronises `stream`. */
+int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stream,
+                    uint32_t *choice);
+
+/* The flags (path | fused/split) that forward would use for M tokens now. */
+int spear_w4ec_dispatch(const spear_w4ec *h, int64_t M, uint32_t *choice);
+
+/* Human-readable name of a status code (static storage). */
+const char *spear_w4ec_strerror(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPEAR_W4EC_H */

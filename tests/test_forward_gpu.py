@@ -1,0 +1,201 @@
+"""Forward pass through the C ABI vs the fp64 oracle, plus bitwise invariants.
+
+Tolerance: see tests/helpers.py (elementwise 1e-2 + 1e-2*|y_ref|, relative
+Frobenius 5e-3).  Configurations follow the Llama-class shapes of the
+workloads (tiny 16x256x256 r8, q/o 4096x4096 r32, MLP 4096x14336 and
+14336x4096 r64, prefill 4096x14336 r64).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from helpers import Problem, assert_close
+
+pytestmark = pytest.mark.gpu
+
+FUSED, SPLIT, DECODE, TC, EC_OFF = 2, 4, 8, 16, 1
+
+
+def _run(P: Problem, flags=0, x=None):
+    torch.cuda.synchronize()
+    y = P.lin(P.xd if x is None else x, flags)
+    torch.cuda.synchronize()
+    assert P.lin.status() == 0
+    return y
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 8, 13, 16])
+def test_tiny_config_all_token_counts(M):
+    P = Problem(M, 256, 256, 8, seed=0, x_outlier_frac=0.0)
+    assert_close(_run(P), P.oracle_y())
+    P.close()
+
+
+@pytest.mark.parametrize("M,K,N,r", [(3, 136, 40, 5), (33, 200, 72, 3), (17, 1032, 264, 20), (40, 64, 8, 1),
+                                     (7, 8, 8, 1), (9, 4104, 136, 33)])
+def test_ragged_shapes(M, K, N, r):
+    P = Problem(M, K, N, r, seed=M + K)
+    for flags in (0, DECODE | FUSED, DECODE | SPLIT):
+        assert_close(_run(P, flags), P.oracle_y(), f"flags={flags}")
+    P.close()
+
+
+@pytest.mark.parametrize("M", [1, 4, 16])
+def test_decode_qo_full_size(M):
+    P = Problem(M, 4096, 4096, 32, seed=0)
+    ref = P.oracle_y()
+    assert_close(_run(P), ref)
+    assert_close(_run(P, DECODE | SPLIT), ref, "split")
+    P.close()
+
+
+@pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096)])
+@pytest.mark.parametrize("M", [1, 16])
+def test_decode_mlp_full_size(M, K, N):
+    P = Problem(M, K, N, 64, seed=0)
+    assert_close(_run(P), P.oracle_y())
+    P.close()
+
+
+@pytest.mark.parametrize("K,N", [(4096, 14336), (14336, 4096)])
+@pytest.mark.parametrize("M", [64, 128])
+def test_decode_mlp_larger_batches_sampled(M, K, N):
+    P = Problem(M, K, N, 64, seed=0)
+    y = _run(P).cpu()
+    rng = np.random.default_rng(M)
+    t = rng.integers(0, M, 3000)
+    n = rng.integers(0, N, 3000)
+    assert_close(y.float()[t, n], P.oracle_sampled(t, n))
+    P.close()
+
+
+def test_ec_isolated_on_qo_shape():
+    """y(EC on) - y(EC off) against the oracle's correction term alone."""
+    P = Problem(16, 4096, 4096, 32, seed=3)
+    y_on = _run(P).double().cpu().numpy()
+    y_off = _run(P, EC_OFF).double().cpu().numpy()
+    ref_on, _, corr = P.oracle_y(want_corr=True)
+    ref_off = ref_on - corr
+    delta = y_on - y_off
+    # two bf16 roundings bound the difference, element by element
+    bound = 2.0 ** -8 * (np.abs(ref_on) + np.abs(ref_off)) + 1e-3 * np.abs(corr) + 1e-6
+    assert np.all(np.abs(delta - corr) <= bound)
+    assert np.linalg.norm(delta - corr) / np.linalg.norm(corr) < 0.1
+    P.close()
+
+
+def test_ec_dominant_variant():
+    """A, B ~ N(0, 1): the correction dominates y, so y's tolerance checks the EC."""
+    P = Problem(16, 4096, 4096, 32, seed=4, ab_std=1.0)
+    ref, _, corr = P.oracle_y(want_corr=True)
+    assert np.linalg.norm(corr) > 10 * np.linalg.norm(ref - corr)
+    assert_close(_run(P), ref)
+    assert_close(_run(P, DECODE | SPLIT), ref, "split")
+    P.close()
+
+
+def test_gate_matches_oracle():
+    P = Problem(37, 4096, 256, 64, seed=5, gate_open_frac=0.3)
+    g = P.lin.gate(P.xd).double().cpu().numpy()
+    import oracle
+    g_ref = oracle.gate(P.x, P.layer.wg, P.layer.b_g)
+    assert np.max(np.abs(g - g_ref)) < 1e-5
+    P.close()
+
+
+def test_gate_closed_and_open_limits():
+    P = Problem(8, 512, 64, 8, seed=6)
+    y_lin = _run(P, EC_OFF)
+    P.lin.close()
+    from w4_gemm_error_b200.spear import W4ECLinear
+    L = P.layer
+    closed = W4ECLinear(L.W.cuda(), L.A.cuda(), L.B.cuda(), L.wg.cuda(), -1e4, max_M=8)
+    assert torch.equal(closed(P.xd), y_lin)          # g == 0 exactly: the plain W4 GEMM
+    closed.close()
+
+
+def test_ec_off_equals_zero_B_and_rank_zero():
+    P = Problem(12, 1024, 384, 16, seed=7)
+    y_off = _run(P, EC_OFF)
+    from w4_gemm_error_b200.spear import W4ECLinear
+    L = P.layer
+    zb = W4ECLinear(L.W.cuda(), L.A.cuda(), torch.zeros_like(L.B).cuda(), L.wg.cuda(), L.b_g, max_M=12)
+    r0 = W4ECLinear(L.W.cuda(), None, None, None, 0.0, max_M=12)
+    assert torch.equal(zb(P.xd), y_off)
+    assert torch.equal(r0(P.xd), y_off)
+    zb.close()
+    r0.close()
+    P.close()
+
+
+def test_invariants_determinism_scaling_permutation():
+    P = Problem(16, 4096, 1024, 32, seed=8)
+    y1 = _run(P)
+    for _ in range(3):
+        assert torch.equal(_run(P), y1), "repeated runs differ"
+    y_off = _run(P, EC_OFF)
+    y2 = _run(P, EC_OFF, x=(P.xd.float() * 2).to(torch.bfloat16))
+    assert torch.equal(y2, (y_off.float() * 2).to(torch.bfloat16)), "y(2x) != 2 y(x)"
+    perm = torch.randperm(16, generator=torch.Generator().manual_seed(0))
+    yp = _run(P, 0, x=P.xd[perm.cuda()].contiguous())
+    assert torch.equal(yp, y1[perm.cuda()]), "token permutation"
+    P.close()
+
+
+def test_host_buffer_entry_matches_device_entry():
+    from w4_gemm_error_b200 import spear
+    P = Problem(9, 1024, 512, 16, seed=9)
+    y_dev = _run(P).cpu()
+    x_h = P.x.clone().pin_memory()
+    y_h = torch.empty((9, 512), dtype=torch.bfloat16).pin_memory()
+    spear.spear_w4ec_forward_host(P.lin.h, x_h, y_h, 9)
+    assert torch.equal(y_h, y_dev)
+    P.close()
+
+
+def test_tune_records_a_legal_choice():
+    P = Problem(16, 4096, 4096, 32, seed=10)
+    y = torch.empty((16, 4096), dtype=torch.bfloat16, device="cuda")
+    choice = P.lin.tune(P.xd, y)
+    assert choice & (DECODE | TC) and choice & (FUSED | SPLIT)
+    assert P.lin.dispatch(16) == choice
+    assert_close(_run(P), P.oracle_y())
+    P.close()
+
+
+def test_argument_errors():
+    from w4_gemm_error_b200 import spear
+    P = Problem(4, 256, 256, 8, seed=11, max_M=4)
+    h = P.lin.h
+    lib = spear.lib()
+    y = torch.empty((8, 256), dtype=torch.bfloat16, device="cuda")
+    x8 = torch.zeros((8, 256), dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    assert lib.spear_w4ec_forward(h, x8.data_ptr(), y.data_ptr(), 8, 0, s) == spear.SPEAR_ERR_INVALID  # M > max_M
+    assert lib.spear_w4ec_forward(h, x8.data_ptr() + 2, y.data_ptr(), 1, 0, s) == spear.SPEAR_ERR_INVALID
+    assert lib.spear_w4ec_forward(h, x8.data_ptr(), y.data_ptr(), 0, 0, s) == spear.SPEAR_OK
+    assert lib.spear_w4ec_forward(h, x8.data_ptr(), y.data_ptr(), 1, DECODE | TC, s) == spear.SPEAR_ERR_INVALID
+    fresh = spear.spear_w4ec_create(256, 256, 8, 4)
+    assert lib.spear_w4ec_forward(fresh, x8.data_ptr(), y.data_ptr(), 1, 0, s) == spear.SPEAR_ERR_STATE
+    spear.spear_w4ec_destroy(fresh)
+    r0 = spear.spear_w4ec_create(256, 256, 0, 4)
+    g = torch.empty(4, device="cuda")
+    assert lib.spear_w4ec_get_gate(r0, x8.data_ptr(), g.data_ptr(), 1, s) == spear.SPEAR_ERR_UNSUPPORTED
+    spear.spear_w4ec_destroy(r0)
+    P.close()
+
+
+def test_injected_faults_are_reported(monkeypatch):
+    from w4_gemm_error_b200 import spear
+    monkeypatch.setenv("SPEAR_FAULT", "alloc")
+    with pytest.raises(spear.SpearError) as ei:
+        spear.spear_w4ec_create(256, 256, 8, 4)
+    assert ei.value.status == spear.SPEAR_ERR_NOMEM
+    monkeypatch.setenv("SPEAR_FAULT", "launch")
+    P = Problem(4, 256, 256, 8, seed=12)
+    with pytest.raises(spear.SpearError) as ei:
+        P.lin(P.xd)
+    assert ei.value.status == spear.SPEAR_ERR_CUDA
+    P.close()

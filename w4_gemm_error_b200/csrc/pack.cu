@@ -1,0 +1,127 @@
+// Per-output-channel round-to-nearest int4 packing of a bf16 weight matrix,
+// and the operand layouts of the Error Compensator.
+//
+// SPEAR, "A System for Post-Quantization Error-Adaptive Recovery Enabling
+// Efficient Low-Bit LLM Serving", Abstract: weights are held at 4 bits per
+// output channel.  The rounding rule and bit layout are this library's
+// reading (the pages give neither):
+//   s[n] = fp32(max_k |W[n,k]|) / 7        (IEEE fp32 division)
+//   q    = clamp(rint(fp32(W[n,k] / s[n])), -8, 7) + 8    (ties to even)
+//   z[n] = 8;  an all-zero row has s = 0 and every code 8
+//   code of k = 8j+i in bits [4i, 4i+3] of word j of row n.
+#include "device_utils.cuh"
+#include "kernels.h"
+
+namespace spear {
+namespace {
+
+constexpr int kPackWarps = 8;
+
+__global__ void __launch_bounds__(kPackWarps * 32)
+pack_w4_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K, int64_t Np, int64_t Kp,
+               uint32_t *__restrict__ codes, float *__restrict__ s, uint8_t *__restrict__ z,
+               int *status)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kPackWarps + (threadIdx.x >> 5);
+    if (row >= Np)
+        return;
+    const int64_t words = Kp / 8, valid_words = K / 8;
+    uint32_t *crow = codes + row * words;
+    if (row >= N) {
+        for (int64_t j = lane; j < words; j += 32)
+            crow[j] = 0x88888888u;
+        if (lane == 0) {
+            s[row] = 0.0f;
+            z[row] = 8;
+        }
+        return;
+    }
+    const uint16_t *wrow = W + row * K;
+
+    // pass 1: amax of the row (bf16 -> fp32 is exact), and a non-finite check
+    uint32_t amax_bits = 0;  // |w| as bits: ordered like the values for finite inputs
+    for (int64_t j = lane; j < valid_words; j += 32) {
+        const uint4 v = ld_nc(wrow + 8 * j);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            amax_bits = max(amax_bits, (w4[i] & 0x7FFFu) << 16);
+            amax_bits = max(amax_bits, w4[i] & 0x7FFF0000u);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        amax_bits = max(amax_bits, __shfl_xor_sync(0xFFFFFFFFu, amax_bits, o));
+    if (amax_bits >= 0x7F800000u && lane == 0)
+        atomicOr(status, kStatusNonFinite);
+    const float amax = __uint_as_float(amax_bits);
+    const float sn = __fdiv_rn(amax, 7.0f);
+
+    // pass 2: quantise and pack eight codes per word
+    for (int64_t j = lane; j < words; j += 32) {
+        uint32_t word = 0x88888888u;
+        if (j < valid_words && sn != 0.0f) {
+            const uint4 v = ld_nc(wrow + 8 * j);
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            word = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t h = (i & 1) ? (w4[i >> 1] & 0xFFFF0000u) : (w4[i >> 1] << 16);
+                float c = rintf(__fdiv_rn(__uint_as_float(h), sn));
+                c = fminf(fmaxf(c, -8.0f), 7.0f);
+                word |= (uint32_t)((int)c + 8) << (4 * i);
+            }
+        }
+        crow[j] = word;
+    }
+    if (lane == 0) {
+        s[row] = sn;
+        z[row] = 8;
+    }
+}
+
+// G [R1p][Kp]: row 0 = w_g, rows 1..r = A^T;  Bt [Np][rp] = B^T; zeros elsewhere.
+__global__ void pack_ec_kernel(const uint16_t *__restrict__ A, const uint16_t *__restrict__ B,
+                               const uint16_t *__restrict__ wg, int64_t K, int64_t N, int r,
+                               int64_t Kp, int64_t Np, int R1p, int rp, uint16_t *__restrict__ G,
+                               uint16_t *__restrict__ Bt)
+{
+    const int64_t nG = (int64_t)R1p * Kp, nB = Np * rp;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nG + nB;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < nG) {
+            const int64_t j = i / Kp, k = i - j * Kp;
+            uint16_t v = 0;
+            if (k < K) {
+                if (j == 0)
+                    v = wg[k];
+                else if (j - 1 < r)
+                    v = A[k * r + (j - 1)];
+            }
+            G[i] = v;
+        } else {
+            const int64_t e = i - nG, n = e / rp, j = e - n * rp;
+            Bt[e] = (n < N && j < r) ? B[j * N + n] : (uint16_t)0;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_pack(const Packed &pk, const void *W, const void *A, const void *B,
+                        const void *wg, int *status, cudaStream_t st)
+{
+    const int blocks = (int)((pk.Np + kPackWarps - 1) / kPackWarps);
+    pack_w4_kernel<<<blocks, kPackWarps * 32, 0, st>>>(static_cast<const uint16_t *>(W), pk.N, pk.K,
+                                                       pk.Np, pk.Kp, pk.codes, pk.s, pk.z, status);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || pk.r == 0)
+        return e;
+    pack_ec_kernel<<<1024, 256, 0, st>>>(static_cast<const uint16_t *>(A), static_cast<const uint16_t *>(B),
+                                         static_cast<const uint16_t *>(wg), pk.K, pk.N, pk.r, pk.Kp, pk.Np,
+                                         pk.R1p, pk.rp, pk.G, pk.Bt);
+    return cudaGetLastError();
+}
+
+}  // namespace spear

@@ -1,0 +1,252 @@
+// Per-token gate and Error Compensator down-projection.
+//
+// SPEAR, "A System for Post-Quantization Error-Adaptive Recovery Enabling
+// Efficient Low-Bit LLM Serving", Abstract: the EC is "modulated by
+// per-token gates".  This library's reading of that gate and of the EC:
+//   logit_t = x[t,:] . w_g + b_g,   g_t = 1 / (1 + exp(-logit_t))
+//   u[t,j]  = x[t,:] . A[:,j]       v[t,j] = bf16(g_t * u[t,j])
+// v is the left operand of the EC up-projection that the GEMM kernels add
+// to their accumulators (y += v . B).
+//
+// Both dot products are one small GEMM, D[j][t] = G[j,:] . x[t,:] with
+// G = [w_g; A^T] (R1p rows), run on the tensor cores with mma.sync: G rows on
+// the 16-row side, 16 tokens per CTA on the 8-column side, the K range split
+// over the CTA's four warps and, when few tokens leave SMs idle, over CTAs.
+// Split-K partials are summed in a fixed order by the last CTA of each token
+// tile to arrive (no floating-point atomics, run-to-run identical).
+#include <algorithm>
+
+#include "device_utils.cuh"
+#include "kernels.h"
+
+namespace spear {
+namespace {
+
+constexpr int kTok = 16;  // tokens per CTA (two 8-column MMA tiles)
+
+struct PrepassParams {
+    const uint16_t *G;
+    const uint16_t *x;
+    int64_t M, K, Kp;
+    int R1p, r, rp;
+    float b_g;
+    int S;       // CTAs per token tile (split-K)
+    int bps;     // 64-wide k blocks per split
+    uint16_t *v;
+    float *g;
+    float *part;
+    unsigned *counters;
+};
+
+template <int MT>
+__global__ void __launch_bounds__(128) prepass_kernel(PrepassParams p)
+{
+    pdl_launch_dependents();
+    pdl_wait();  // x is written by the previous kernel in the stream
+    extern __shared__ float4 smem_f4[];
+    float *red = reinterpret_cast<float *>(smem_f4);  // [4][R1p][kTok]
+    __shared__ int s_last;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, c = lane & 3;
+    const int tile = blockIdx.x / p.S, ks = blockIdx.x - tile * p.S;
+    const int64_t t0 = (int64_t)tile * kTok;
+    const int nkb = (int)(p.Kp / 64);
+    const int kb0 = ks * p.bps, kb1 = min(kb0 + p.bps, nkb);
+
+    float acc[MT][2][4];
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                acc[m][n][i] = 0.f;
+
+    for (int kb = kb0 + warp; kb < kb1; kb += 4) {
+        const int64_t k = (int64_t)kb * 64 + 16 * c;
+        uint32_t xb[2][8];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            const int64_t t = t0 + 8 * n + gid;
+            uint4 a = make_uint4(0, 0, 0, 0), b = a;
+            if (t < p.M && k < p.K) {
+                const uint16_t *src = p.x + t * p.K + k;
+                a = ld_nc(src);
+                if (k + 8 < p.K)
+                    b = ld_nc(src + 8);
+            }
+            xb[n][0] = a.x; xb[n][1] = a.y; xb[n][2] = a.z; xb[n][3] = a.w;
+            xb[n][4] = b.x; xb[n][5] = b.y; xb[n][6] = b.z; xb[n][7] = b.w;
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+            const uint16_t *g0 = p.G + (int64_t)(16 * m + gid) * p.Kp + k;
+            const uint16_t *g1 = g0 + 8 * p.Kp;
+            const uint4 a0 = ld_nc(g0), a1 = ld_nc(g0 + 8), h0 = ld_nc(g1), h1 = ld_nc(g1 + 8);
+            const uint32_t ga[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const uint32_t ha[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
+            // step i covers k = 16c + 4i + {0,1} (first pair) and + {2,3} (second pair)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int n = 0; n < 2; ++n)
+                    mma_bf16_16816(acc[m][n], ga[2 * i], ha[2 * i], ga[2 * i + 1], ha[2 * i + 1],
+                                   xb[n][2 * i], xb[n][2 * i + 1]);
+        }
+    }
+
+    // reduce the four warps' partial tiles through shared memory
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+            float *base = red + ((size_t)warp * p.R1p) * kTok;
+            const int r0 = 16 * m + gid, col = 8 * n + 2 * c;
+            base[r0 * kTok + col] = acc[m][n][0];
+            base[r0 * kTok + col + 1] = acc[m][n][1];
+            base[(r0 + 8) * kTok + col] = acc[m][n][2];
+            base[(r0 + 8) * kTok + col + 1] = acc[m][n][3];
+        }
+    __syncthreads();
+    const int tile_elems = p.R1p * kTok;
+    for (int e = tid; e < tile_elems; e += 128)
+        red[e] = red[e] + red[tile_elems + e] + red[2 * tile_elems + e] + red[3 * tile_elems + e];
+    __syncthreads();
+
+    if (p.S > 1) {
+        float *mine = p.part + ((size_t)tile * p.S + ks) * tile_elems;
+        for (int e = tid; e < tile_elems; e += 128)
+            mine[e] = red[e];
+        __threadfence();
+        __syncthreads();
+        if (tid == 0)
+            s_last = (atomicAdd(&p.counters[tile], 1u) == (unsigned)(p.S - 1));
+        __syncthreads();
+        if (!s_last)
+            return;
+        __threadfence();
+        const float *all = p.part + (size_t)tile * p.S * tile_elems;
+        for (int e = tid; e < tile_elems; e += 128) {
+            float sum = 0.f;
+            for (int q = 0; q < p.S; ++q)
+                sum += __ldcg(all + (size_t)q * tile_elems + e);
+            red[e] = sum;
+        }
+        if (tid == 0)
+            p.counters[tile] = 0u;
+        __syncthreads();
+    }
+
+    // epilogue: gate and v for the tile's tokens (row 0 of the tile is the logit)
+    __shared__ float s_gate[kTok];
+    if (tid < kTok) {
+        const float gt = 1.0f / (1.0f + expf(-(red[tid] + p.b_g)));
+        s_gate[tid] = gt;
+        if (t0 + tid < p.M)
+            p.g[t0 + tid] = gt;
+    }
+    __syncthreads();
+    for (int e = tid; e < kTok * p.rp; e += 128) {
+        const int tt = e / p.rp, j = e - tt * p.rp;
+        const int64_t t = t0 + tt;
+        if (t >= p.M)
+            continue;
+        const float val = (j < p.r) ? s_gate[tt] * red[(1 + j) * kTok + tt] : 0.f;
+        p.v[t * p.rp + j] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+    }
+}
+
+int pick_splits(int64_t M, int64_t Kp, int num_sms)
+{
+    const int tiles = (int)((M + kTok - 1) / kTok);
+    const int nkb = (int)(Kp / 64);
+    int S = std::max(1, (2 * num_sms) / std::max(tiles, 1));
+    S = std::min(S, std::max(1, nkb / 4));  // at least one k block per warp
+    return std::min(S, 64);
+}
+
+using PrepassFn = void (*)(PrepassParams);
+PrepassFn prepass_fn(int MT)
+{
+    switch (MT) {
+    case 1: return prepass_kernel<1>;
+    case 2: return prepass_kernel<2>;
+    case 3: return prepass_kernel<3>;
+    case 4: return prepass_kernel<4>;
+    case 5: return prepass_kernel<5>;
+    case 6: return prepass_kernel<6>;
+    case 7: return prepass_kernel<7>;
+    case 8: return prepass_kernel<8>;
+    case 9: return prepass_kernel<9>;
+    default: return nullptr;
+    }
+}
+
+}  // namespace
+
+size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms)
+{
+    size_t worst = 0;
+    // the split count shrinks as M grows; check every tile count up to max_M
+    const int64_t tiles_max = (max_M + kTok - 1) / kTok;
+    for (int64_t tiles = 1; tiles <= tiles_max; ++tiles) {
+        const int S = pick_splits(tiles * kTok, pk.Kp, num_sms);
+        if (S > 1)
+            worst = std::max(worst, (size_t)tiles * S * pk.R1p * kTok);
+        else
+            break;
+    }
+    return worst;
+}
+
+int prepass_counters(int64_t max_M) { return (int)((max_M + kTok - 1) / kTok); }
+
+cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t *v, float *g,
+                           const PrepassWork &w, cudaStream_t st, int num_sms)
+{
+    if (M <= 0 || pk.r == 0)
+        return cudaSuccess;
+    PrepassParams p;
+    p.G = pk.G;
+    p.x = static_cast<const uint16_t *>(x);
+    p.M = M;
+    p.K = pk.K;
+    p.Kp = pk.Kp;
+    p.R1p = pk.R1p;
+    p.r = pk.r;
+    p.rp = pk.rp;
+    p.b_g = pk.b_g;
+    p.S = pick_splits(M, pk.Kp, num_sms);
+    const int nkb = (int)(pk.Kp / 64);
+    p.bps = (nkb + p.S - 1) / p.S;
+    p.S = (nkb + p.bps - 1) / p.bps;  // drop empty splits
+    p.v = v;
+    p.g = g;
+    p.part = w.part;
+    p.counters = w.counters;
+    const int tiles = (int)((M + kTok - 1) / kTok);
+    if (tiles > w.n_counters || (p.S > 1 && (size_t)tiles * p.S * pk.R1p * kTok > w.part_floats))
+        return cudaErrorInvalidValue;
+    PrepassFn fn = prepass_fn(pk.R1p / 16);
+    if (!fn)
+        return cudaErrorInvalidValue;
+    const size_t smem = (size_t)4 * pk.R1p * kTok * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = raise_smem_limit(reinterpret_cast<const void *>(fn), smem);
+        if (e != cudaSuccess)
+            return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(tiles * p.S));
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fn, p);
+}
+
+}  // namespace spear

@@ -1,0 +1,225 @@
+"""Python binding of libspear_w4ec (ctypes): argument marshalling only.
+
+Every function here has the name of the C entry point it calls
+(include/spear_w4ec.h) and does no arithmetic of its own: PyTorch provides
+device memory and streams, the library's kernels do all the work.  If the
+shared library is missing or fails to load, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspear_w4ec.so")
+
+SPEAR_OK = 0
+SPEAR_ERR_INVALID = -1
+SPEAR_ERR_UNSUPPORTED = -2
+SPEAR_ERR_NOMEM = -3
+SPEAR_ERR_CUDA = -4
+SPEAR_ERR_TIMEOUT = -5
+SPEAR_ERR_DEVICE = -6
+SPEAR_ERR_STATE = -7
+
+SPEAR_EC_OFF = 1
+SPEAR_FORCE_FUSED = 2
+SPEAR_FORCE_SPLIT = 4
+SPEAR_FORCE_DECODE = 8
+SPEAR_FORCE_TC = 16
+
+EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_forward", "spear_w4ec_forward_host",
+            "spear_w4ec_destroy", "spear_w4ec_get_packed", "spear_w4ec_get_gate", "spear_w4ec_sync_status",
+            "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_strerror")
+
+
+class SpearError(RuntimeError):
+    def __init__(self, status: int, call: str):
+        self.status = status
+        super().__init__(f"{call}: {strerror(status)} ({status})")
+
+
+class _Opts(ctypes.Structure):
+    _fields_ = [("max_M", ctypes.c_int64), ("device", ctypes.c_int32)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m w4_gemm_error_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, u32, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_float
+    sig = {
+        "spear_w4ec_create": [ctypes.POINTER(P), i64, i64, i32, ctypes.POINTER(_Opts)],
+        "spear_w4ec_pack": [P, P, P, P, P, f32, P],
+        "spear_w4ec_forward": [P, P, P, i64, u32, P],
+        "spear_w4ec_forward_host": [P, P, P, i64, u32, P],
+        "spear_w4ec_destroy": [P],
+        "spear_w4ec_get_packed": [P, P, P, P, P],
+        "spear_w4ec_get_gate": [P, P, P, i64, P],
+        "spear_w4ec_sync_status": [P, P],
+        "spear_w4ec_tune": [P, P, P, i64, P, ctypes.POINTER(u32)],
+        "spear_w4ec_dispatch": [P, i64, ctypes.POINTER(u32)],
+    }
+    for name, args in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = ctypes.c_int
+    lib.spear_w4ec_strerror.argtypes = [ctypes.c_int]
+    lib.spear_w4ec_strerror.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+def lib():
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return _lib.spear_w4ec_strerror(int(status)).decode()
+
+
+def _check(rc: int, call: str):
+    if rc != SPEAR_OK:
+        raise SpearError(rc, call)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        return ctypes.c_void_p(t.data_ptr())
+    return ctypes.c_void_p(int(t))
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev_bf16(t: torch.Tensor, shape, name):
+    if not (t.is_cuda and t.dtype == torch.bfloat16 and t.is_contiguous() and tuple(t.shape) == tuple(shape)):
+        raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape {tuple(shape)}")
+
+
+def spear_w4ec_create(K: int, N: int, r: int, max_M: int = 4096, device: int = -1) -> int:
+    h = ctypes.c_void_p()
+    opts = _Opts(max_M, device)
+    _check(_lib.spear_w4ec_create(ctypes.byref(h), K, N, r, ctypes.byref(opts)), "spear_w4ec_create")
+    return h.value
+
+
+def spear_w4ec_pack(h: int, W, A, B, w_g, b_g: float, stream=None):
+    _check(_lib.spear_w4ec_pack(h, _ptr(W), _ptr(A), _ptr(B), _ptr(w_g), float(b_g), _stream(stream)),
+           "spear_w4ec_pack")
+
+
+def spear_w4ec_forward(h: int, x, y, M: int, flags: int = 0, stream=None):
+    _check(_lib.spear_w4ec_forward(h, _ptr(x), _ptr(y), M, flags, _stream(stream)), "spear_w4ec_forward")
+
+
+def spear_w4ec_forward_host(h: int, x_host, y_host, M: int, flags: int = 0, stream=None):
+    _check(_lib.spear_w4ec_forward_host(h, _ptr(x_host), _ptr(y_host), M, flags, _stream(stream)),
+           "spear_w4ec_forward_host")
+
+
+def spear_w4ec_destroy(h: int):
+    _check(_lib.spear_w4ec_destroy(h), "spear_w4ec_destroy")
+
+
+def spear_w4ec_get_packed(h: int, codes=None, s=None, z=None, stream=None):
+    _check(_lib.spear_w4ec_get_packed(h, _ptr(codes), _ptr(s), _ptr(z), _stream(stream)), "spear_w4ec_get_packed")
+
+
+def spear_w4ec_get_gate(h: int, x, g, M: int, stream=None):
+    _check(_lib.spear_w4ec_get_gate(h, _ptr(x), _ptr(g), M, _stream(stream)), "spear_w4ec_get_gate")
+
+
+def spear_w4ec_sync_status(h: int, stream=None) -> int:
+    return int(_lib.spear_w4ec_sync_status(h, _stream(stream)))
+
+
+def spear_w4ec_tune(h: int, x, y, M: int, stream=None) -> int:
+    choice = ctypes.c_uint32(0)
+    _check(_lib.spear_w4ec_tune(h, _ptr(x), _ptr(y), M, _stream(stream), ctypes.byref(choice)), "spear_w4ec_tune")
+    return choice.value
+
+
+def spear_w4ec_dispatch(h: int, M: int) -> int:
+    choice = ctypes.c_uint32(0)
+    _check(_lib.spear_w4ec_dispatch(h, M, ctypes.byref(choice)), "spear_w4ec_dispatch")
+    return choice.value
+
+
+class W4ECLinear:
+    """Owning wrapper of one packed layer (create + pack; destroy on close).
+
+    Shapes: W [N, K], A [K, r], B [r, N], w_g [K] (bf16 CUDA tensors).
+    """
+
+    def __init__(self, W: torch.Tensor, A: torch.Tensor | None, B: torch.Tensor | None,
+                 w_g: torch.Tensor | None, b_g: float, max_M: int = 4096, stream=None):
+        N, K = W.shape
+        r = 0 if A is None else A.shape[1]
+        _dev_bf16(W, (N, K), "W")
+        if r:
+            _dev_bf16(A, (K, r), "A")
+            _dev_bf16(B, (r, N), "B")
+            _dev_bf16(w_g, (K,), "w_g")
+        self.K, self.N, self.r, self.max_M = K, N, r, max_M
+        self.device = W.device
+        self.h = spear_w4ec_create(K, N, r, max_M, W.device.index if W.device.index is not None else -1)
+        try:
+            spear_w4ec_pack(self.h, W, A, B, w_g, b_g, stream)
+        except Exception:
+            spear_w4ec_destroy(self.h)
+            self.h = None
+            raise
+
+    def forward(self, x: torch.Tensor, flags: int = 0, out: torch.Tensor | None = None, stream=None):
+        M = x.shape[0]
+        _dev_bf16(x, (M, self.K), "x")
+        y = out if out is not None else torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device)
+        _dev_bf16(y, (M, self.N), "y")
+        spear_w4ec_forward(self.h, x, y, M, flags, stream)
+        return y
+
+    __call__ = forward
+
+    def packed(self, stream=None):
+        codes = torch.empty((self.N, self.K // 8), dtype=torch.int32, device=self.device)
+        s = torch.empty(self.N, dtype=torch.float32, device=self.device)
+        z = torch.empty(self.N, dtype=torch.uint8, device=self.device)
+        spear_w4ec_get_packed(self.h, codes, s, z, stream)
+        return codes, s, z
+
+    def gate(self, x: torch.Tensor, stream=None):
+        M = x.shape[0]
+        _dev_bf16(x, (M, self.K), "x")
+        g = torch.empty(M, dtype=torch.float32, device=x.device)
+        spear_w4ec_get_gate(self.h, x, g, M, stream)
+        return g
+
+    def status(self, stream=None) -> int:
+        return spear_w4ec_sync_status(self.h, stream)
+
+    def tune(self, x: torch.Tensor, y: torch.Tensor, stream=None) -> int:
+        return spear_w4ec_tune(self.h, x, y, x.shape[0], stream)
+
+    def dispatch(self, M: int) -> int:
+        return spear_w4ec_dispatch(self.h, M)
+
+    def close(self):
+        if getattr(self, "h", None):
+            spear_w4ec_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
