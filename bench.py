@@ -274,7 +274,7 @@ def run_ours(args, rank, world, local_rank):
     if wl["kind"] == "decode":
         roof = {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": round(per_gpu / peaks["hbm"], 4), "traffic": None,
-                "kernel": "decode_w4ec_kernel (+ prepass overlapped by PDL): per-forward time",
+                "kernel": "decode_w4ec_kernel (one launch per forward): per-forward time in the chained stack",
                 "peak_source": peaks["source"]}
     else:
         pk = peaks["bf16_sustained"]
@@ -286,7 +286,8 @@ def run_ours(args, rank, world, local_rank):
     for M in Ms:
         ch = layers[0].dispatch(M)
         if ch & spear.SPEAR_FORCE_DECODE:
-            n = math.ceil(M / 32) + (1 if r else 0) + (1 if (r and ch & spear.SPEAR_FORCE_SPLIT) else 0)
+            split = bool(r and ch & spear.SPEAR_FORCE_SPLIT)
+            n = math.ceil(M / 32) + (2 if split else 0)   # split: prepass + separate EC kernel
         else:
             n = 1 + (1 if r else 0) + (1 if (r and ch & spear.SPEAR_FORCE_SPLIT) else 0)
         launches_per_forward[M] = n

@@ -76,23 +76,44 @@ def test_ec_isolated_on_qo_shape():
     P = Problem(16, 4096, 4096, 32, seed=3)
     y_on = _run(P).double().cpu().numpy()
     y_off = _run(P, EC_OFF).double().cpu().numpy()
-    ref_on, _, corr = P.oracle_y(want_corr=True)
+    ref_on, g, corr = P.oracle_y(want_corr=True)
     ref_off = ref_on - corr
     delta = y_on - y_off
-    # two bf16 roundings bound the difference, element by element
-    bound = 2.0 ** -8 * (np.abs(ref_on) + np.abs(ref_off)) + 1e-3 * np.abs(corr) + 1e-6
+    # Error budget of delta - corr, element by element: the two bf16 roundings
+    # of y (unit roundoff 2^-8 each) and the bf16 rounding of v = g*(x.A)
+    # (2^-8 of each term of sum_j v_j B_j); the main product is computed the
+    # same way with and without the EC, so its fp32 error cancels.
+    xd = P.x.double().numpy()
+    terms = g[:, None] * (np.abs(xd @ P.layer.A.double().numpy()) @ np.abs(P.layer.B.double().numpy()))
+    bound = 2.0 ** -8 * (np.abs(ref_on) + np.abs(ref_off) + terms) + 1e-4 * terms + 1e-6
     assert np.all(np.abs(delta - corr) <= bound)
-    assert np.linalg.norm(delta - corr) / np.linalg.norm(corr) < 0.1
+    # in aggregate the difference tracks the correction (bf16 rounding of y
+    # alone leaves about 10% relative noise at this correction size)
+    assert np.linalg.norm(delta - corr) / np.linalg.norm(corr) < 0.25
     P.close()
 
 
 def test_ec_dominant_variant():
-    """A, B ~ N(0, 1): the correction dominates y, so y's tolerance checks the EC."""
+    """A, B ~ N(0, 1): the correction dominates y, so y's tolerance checks the EC.
+
+    The fused decode kernel keeps v = g*(x.A) in fp32 and meets the plain
+    tolerance.  The split path rounds the plain GEMM's output to bf16 before
+    adding the correction (2^-8 of |main| more where main and correction
+    cancel); the tcgen05 kernel feeds v and B^T/s to the tensor cores as
+    bf16 (up to 2^-8 of |v_j B_j| per term for each of the two roundings).
+    Their bounds add those terms to the plain tolerance.
+    """
     P = Problem(16, 4096, 4096, 32, seed=4, ab_std=1.0)
-    ref, _, corr = P.oracle_y(want_corr=True)
+    ref, g, corr = P.oracle_y(want_corr=True)
     assert np.linalg.norm(corr) > 10 * np.linalg.norm(ref - corr)
     assert_close(_run(P), ref)
-    assert_close(_run(P, DECODE | SPLIT), ref, "split")
+    y_split = _run(P, DECODE | SPLIT).double().cpu().numpy()
+    assert np.all(np.abs(y_split - ref) <= 1e-2 + 1e-2 * np.abs(ref) + 2.0 ** -8 * np.abs(ref - corr))
+    xd = P.x.double().numpy()
+    terms = g[:, None] * (np.abs(xd @ P.layer.A.double().numpy()) @ np.abs(P.layer.B.double().numpy()))
+    y_tc = _run(P, TC | FUSED).double().cpu().numpy()
+    assert np.all(np.abs(y_tc - ref) <= 1e-2 + 1e-2 * np.abs(ref) + 2.0 ** -7 * terms)
+    assert np.linalg.norm(y_tc - ref) / np.linalg.norm(ref) < 5e-3
     P.close()
 
 
@@ -198,4 +219,61 @@ def test_injected_faults_are_reported(monkeypatch):
     with pytest.raises(spear.SpearError) as ei:
         P.lin(P.xd)
     assert ei.value.status == spear.SPEAR_ERR_CUDA
+    P.close()
+
+
+# ------------------------------------------------------------------ tcgen05 tile kernel
+
+@pytest.mark.parametrize("M,K,N,r", [(33, 256, 128, 8), (256, 4096, 1024, 64), (300, 512, 256, 32),
+                                     (1000, 1032, 264, 20), (513, 4104, 136, 33), (64, 2048, 512, 32),
+                                     (9, 8, 8, 1), (700, 8192, 256, 128)])
+def test_tc_path_shapes(M, K, N, r):
+    P = Problem(M, K, N, r, seed=M + N)
+    ref = P.oracle_y()
+    for flags in (TC | FUSED, TC | SPLIT):
+        assert_close(_run(P, flags), ref, f"flags={flags}")
+    assert_close(_run(P, TC | EC_OFF), P.oracle_y(ec_on=False), "EC off")
+    P.close()
+
+
+def test_tc_path_invariants():
+    P = Problem(300, 1024, 512, 32, seed=13)
+    y1 = _run(P, TC)
+    assert torch.equal(_run(P, TC), y1), "repeated runs differ"
+    y_off = _run(P, TC | EC_OFF)
+    y2 = _run(P, TC | EC_OFF, x=(P.xd.float() * 2).to(torch.bfloat16))
+    assert torch.equal(y2, (y_off.float() * 2).to(torch.bfloat16)), "y(2x) != 2 y(x)"
+    perm = torch.randperm(300, generator=torch.Generator().manual_seed(1))
+    yp = _run(P, TC, x=P.xd[perm.cuda()].contiguous())
+    assert torch.equal(yp, y1[perm.cuda()]), "token permutation"
+    P.close()
+
+
+def test_tc_ec_isolated():
+    P = Problem(256, 4096, 1024, 64, seed=14)
+    y_on = _run(P, TC).double().cpu().numpy()
+    y_off = _run(P, TC | EC_OFF).double().cpu().numpy()
+    ref_on, g, corr = P.oracle_y(want_corr=True)
+    ref_off = ref_on - corr
+    xd = P.x.double().numpy()
+    terms = g[:, None] * (np.abs(xd @ P.layer.A.double().numpy()) @ np.abs(P.layer.B.double().numpy()))
+    # two bf16 roundings of y, and the bf16 operands v and B^T/s of the EC
+    bound = 2.0 ** -8 * (np.abs(ref_on) + np.abs(ref_off)) + 2.0 ** -7 * terms + 1e-4 * terms + 1e-6
+    assert np.all(np.abs((y_on - y_off) - corr) <= bound)
+    P.close()
+
+
+@pytest.mark.parametrize("M", [2048, 4096])
+def test_prefill_full_size_sampled(M):
+    """Prefill MLP gate/up shape, heavy rows and ~30% open gates: sampled outputs."""
+    P = Problem(M, 4096, 14336, 64, seed=0, w_row_outlier_frac=0.005, gate_open_frac=0.3)
+    y = _run(P).float().cpu()
+    rng = np.random.default_rng(M)
+    t = rng.integers(0, M, 2000)
+    n = rng.integers(0, 14336, 2000)
+    assert_close(y[t, n], P.oracle_sampled(t, n))
+    # every row of y is finite and the gate opened for about 30% of tokens
+    assert torch.isfinite(y).all()
+    g = P.lin.gate(P.xd).cpu().numpy()
+    assert 0.25 <= float(np.mean(g > 0.5)) <= 0.35
     P.close()

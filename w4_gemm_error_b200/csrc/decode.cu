@@ -1,113 +1,162 @@
-// Decode-size W4 GEMM with the Error Compensator fused into its epilogue.
+// Decode-size W4 GEMM (a few tokens) with the Error Compensator fused in.
 //
 // SPEAR, "A System for Post-Quantization Error-Adaptive Recovery Enabling
 // Efficient Low-Bit LLM Serving", Abstract: the post-EC computation is fused
-// into the low-bit GEMM.  For a few tokens the GEMM is bound by reading the
-// int4 codes from HBM, so this kernel is built around streaming them:
+// into the low-bit GEMM.  For a few tokens the layer is bound by reading the
+// int4 codes from HBM, and in a decode pass its critical path is the chain
+// "previous layer done -> this layer done", so the kernel is built to stream
+// the weights before that chain starts and to keep the chain short:
 //
+//  * one kernel per forward; a cluster of CS CTAs owns 64 weight rows, each
+//    CTA one K/CS slice of them;
+//  * before waiting for the previous kernel (programmatic dependent launch)
+//    every CTA starts TMA copies of its whole slice of codes (and the
+//    cluster's first CTA loads the scales and B^T rows of its epilogue into
+//    registers), so the weight stream overlaps the previous layer; only the
+//    activations are fetched after the wait;
 //  * weight rows sit on the 16-row side of mma.sync m16n8k16 and tokens on
-//    the 8-column side (up to 32 tokens per launch), so one code is read
-//    once however many tokens there are;
-//  * each lane loads 16 bytes (32 codes) of two rows per 128-wide k block
-//    straight from the exported [N][K/8] layout into registers, four blocks
-//    ahead, and dequantises them in registers: two nibbles 16 bits apart
-//    become a bf16x2 pair (q - z) exactly, so the tensor cores see exact
-//    integer weights and the per-channel scale is applied once at the end;
-//  * the k order inside the MMA is permuted so that those register pairs
-//    (codes k and k+4) line up with the activations, which are staged once
-//    per CTA in shared memory (XOR-swizzled, conflict-free) and paired with
-//    one byte-permute per register;
-//  * the K range is split over CTAs; the last CTA of each 64-row block to
-//    finish sums the partial tiles in a fixed order (run-to-run identical)
-//    and runs the epilogue
-//        y[t,n] = bf16( s[n] * acc[t,n] + sum_j v[t,j] * B[j,n] )
-//    where v = g * (x . A) comes from the prepass kernel;
-//  * kernels are chained with programmatic dependent launch: the first code
-//    blocks are requested before waiting for the previous kernel (which
-//    writes x, and v), so the weight stream overlaps the previous kernel's
-//    tail and the prepass.
+//    the 8-column side, so a code is read once for up to 32 tokens; the
+//    codes are dequantised in registers to exact (q - z) bf16 pairs (two
+//    nibbles 16 bits apart per register), and the activations are paired to
+//    match with one byte permute per register, the k order inside the MMA
+//    being permuted accordingly;
+//  * the K split is summed over distributed shared memory inside the
+//    cluster, in rank order (deterministic), with no global round trip;
+//  * the EC down-projection u = x . [w_g, A] runs on R1p/16 extra clusters
+//    of the same grid (the first ones) with the same slicing; they publish u
+//    in global memory behind a counter, and the 64-row clusters read it for
+//    their epilogue
+//        y[t,n] = bf16( s[n] * acc[t,n] + sum_j g_t u[t,j] B[j,n] ),
+//        g_t = 1 / (1 + exp(-(u[t,0] + b_g))),
+//    with a bounded wait (about a second) that records a timeout in the
+//    handle's status word instead of hanging.
 #include <algorithm>
+#include <new>
 
-#include "device_utils.cuh"
+#include "async_utils.cuh"
 #include "kernels.h"
+#include "tensor_map.h"
 
 namespace spear {
 namespace {
 
-constexpr int kRows = 64;      // weight rows per CTA (four warps x 16)
-constexpr int kPrefetch = 4;   // 128-wide k blocks in flight per warp
-constexpr int kMaxBps = 8;     // k blocks per CTA at most (shared-memory bound)
+constexpr int kRows = 64;       // weight rows per cluster (four warps x 16)
+constexpr int kChunk = 256;     // k per code chunk (one 8 KB TMA box of 64 rows)
+constexpr int kMaxChunks = 8;   // so K/CS <= 2048
+constexpr int kUStride = 32;    // token stride of the published u rows
 
-struct DecodeParams {
-    const uint32_t *codes;
-    const float *s;
-    const uint8_t *z;
-    const uint16_t *x;
-    uint16_t *y;
-    const uint16_t *v;
-    const uint16_t *Bt;
-    float *part;
-    unsigned *counters;
-    int64_t M, K, Kp, N;
-    int S, bps, rp;
-    int ec;
+struct Maps {
+    CUtensorMap codes;  // [Np][Kp/8] u32, boxes of 32 words x 64 rows, 128B swizzle
+    CUtensorMap g;      // [R1p][Kp] bf16, boxes of 64 x 16, 128B swizzle
+    CUtensorMap bt;     // [Np][rp] bf16, boxes of rp x 64
 };
 
-__device__ __forceinline__ int swz(int t, int c, int q)
+struct DecodeParams {
+    const uint16_t *Bt;   // [Np][rp]
+    const float *s;
+    const uint8_t *z;
+    uint16_t *y;
+    float *ws_u;          // [R1p][kUStride] fp32
+    unsigned *flags;      // [0] u clusters published, [1] row clusters done with u
+    int *status;
+    int64_t M, N, Kp;
+    int KS, nch;          // k per CTA (a multiple of 256), code chunks per CTA
+    int JB, NC;           // EC clusters, 64-row clusters
+    int r, rp, R1p;
+    float b_g;
+};
+
+struct Smem {
+    uint32_t codes, x, bt, red, u;   // byte offsets from the 1024-aligned base
+    uint32_t total;
+};
+
+template <int TOK>
+__host__ __device__ inline Smem smem_layout(int KS, int rp, int R1p)
 {
-    // physical 16-byte chunk of logical chunk (lane group c, word q) of token t
-    return 4 * c + (q ^ (2 * (c >> 1)) ^ (t & 1));
+    Smem m;
+    m.codes = 0;                                   // 32*KS bytes: codes (64 rows) or G (16 rows bf16)
+    m.x = m.codes + 32 * KS;                       // 2*TOK*KS bytes: activation sub-tiles
+    m.bt = m.x + 2 * TOK * KS;                     // 128*rp bytes: B^T rows of the cluster
+    m.red = m.bt + 128 * rp;                       // 256*TOK bytes: partial tile
+    m.u = m.red + 256 * TOK;                       // u [R1p][TOK], g [TOK], v [TOK][rp] (fp32)
+    m.total = m.u + 4 * R1p * TOK + 4 * TOK * (rp + 1);
+    return m;
+}
+
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity)
+{
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > kWaitBudgetNs)
+            return false;
+    return true;
 }
 
 template <int T>
-__global__ void __launch_bounds__(128) decode_w4ec_kernel(DecodeParams p)
+__global__ void __launch_bounds__(128)
+decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_g,
+                   const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_x,
+                   DecodeParams p, int CS)
 {
     constexpr int TOK = 8 * T;
-    extern __shared__ uint4 smem_u4[];
-    __shared__ int s_last;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[kMaxChunks + 2];
+    __shared__ int s_ok;
 
     pdl_launch_dependents();
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, c = lane & 3;
-    const int nb = blockIdx.x / p.S, ks = blockIdx.x - nb * p.S;
-    const int nkb = (int)(p.Kp / 128);
-    const int kb0 = ks * p.bps, kb1 = min(kb0 + p.bps, nkb);
-    const int nblk = kb1 - kb0;
-    const int64_t words = p.Kp / 8;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, cl = lane & 3;
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t *const bp = smem_raw + (base - raw);
+    const Smem L = smem_layout<TOK>(p.KS, p.rp, p.R1p);
+    const uint32_t rank = cluster_ctarank();
+    const int cluster = blockIdx.x / CS;
+    const bool is_u = cluster < p.JB;
+    const int k0 = (int)rank * p.KS;
+    // the last ranks may hold a shorter (or empty) slice when K/256 is not a multiple of CS
+    const int nch = max(0, min(p.nch, (int)((p.Kp - k0) / kChunk)));
+    const int nsub = 4 * nch;
+    const uint32_t bar_chunk = smem_addr(&bars[0]);
+    const uint32_t bar_x = smem_addr(&bars[kMaxChunks]);
+    const uint32_t bar_bt = smem_addr(&bars[kMaxChunks + 1]);
+    const int n0 = is_u ? 0 : (cluster - p.JB) * kRows;
 
-    // ---- start the code stream first: rows (gid) and (gid + 8) of this warp
-    const int64_t row_g = (int64_t)nb * kRows + warp * 16 + gid;
-    const uint32_t *cg = p.codes + row_g * words + 16 * kb0 + 4 * c;
-    const uint32_t *ch = cg + 8 * words;
-    uint4 wg[kPrefetch], wh[kPrefetch];
+    // epilogue operands of this thread's row, requested before anything else
+    float s_epi = 0.f;
+    uint4 bt_pre[8];
+    if (!is_u && rank == 0) {
+        const int64_t n_epi = n0 + (tid & (kRows - 1));
+        s_epi = __ldg(p.s + n_epi);
 #pragma unroll
-    for (int i = 0; i < kPrefetch; ++i) {
-        if (i < nblk) {
-            wg[i] = ld_stream(cg + 16 * i);
-            wh[i] = ld_stream(ch + 16 * i);
-        }
+        for (int q = 0; q < 8; ++q)
+            bt_pre[q] = (8 * q < p.rp) ? ld_nc(p.Bt + n_epi * p.rp + 8 * q) : make_uint4(0, 0, 0, 0);
     }
-    const uint32_t zg = 128u + p.z[row_g], zh = 128u + p.z[row_g + 8];
-    // bf16 of -(128 + z): exact (an integer below 256)
-    const uint32_t nbg = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)zg));
-    const uint32_t nbh = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)zh));
-    const uint32_t negg = nbg | (nbg << 16), negh = nbh | (nbh << 16);
-
-    // x (and v) are written by the kernels before this one in the stream:
-    // everything above only touched the packed weights.
-    pdl_wait();
-
-    // ---- stage the activations of this k range: [TOK][nblk][16 chunks]
-    uint4 *xs = smem_u4;
-    const int cpt = nblk * 16;
-    for (int i = tid; i < TOK * cpt; i += 128) {
-        const int t = i / cpt, rem = i - t * cpt, b = rem >> 4, chk = rem & 15;
-        const int64_t k = (int64_t)(kb0 + b) * 128 + 8 * chk;
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (t < p.M && k < p.K)
-            val = ld_nc(p.x + (int64_t)t * p.K + k);
-        xs[(t * nblk + b) * 16 + swz(t, chk >> 2, chk & 3)] = val;
+    if (tid == 0) {
+        for (int c = 0; c < kMaxChunks + 2; ++c)
+            mbar_init(bar_chunk + 8 * c, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        // the weights do not depend on earlier kernels: start them now
+        for (int c = 0; c < nch; ++c) {
+            const uint32_t bar = bar_chunk + 8 * c;
+            mbar_expect_tx(bar, 8192);
+            if (is_u) {
+                for (int i = 0; i < 4; ++i)
+                    tma_load_2d(base + L.codes + c * 8192 + i * 2048, &tm_g, k0 + c * kChunk + i * 64, 16 * cluster,
+                                bar);
+            } else {
+                tma_load_2d(base + L.codes + c * 8192, &tm_codes, (k0 + c * kChunk) / 8, n0, bar);
+            }
+        }
+        // the activations are written by the previous kernel in the stream
+        pdl_wait();
+        mbar_expect_tx(bar_x, 2 * TOK * kChunk * nch);
+        for (int i = 0; i < nsub; ++i)
+            tma_load_2d(base + L.x + i * (TOK * 128), &tm_x, k0 + 64 * i, 0, bar_x);
     }
     __syncthreads();
+
+    bool ok = wait_bounded(bar_x, 0);
 
     float acc[T][4];
 #pragma unroll
@@ -116,185 +165,358 @@ __global__ void __launch_bounds__(128) decode_w4ec_kernel(DecodeParams p)
         for (int i = 0; i < 4; ++i)
             acc[n][i] = 0.f;
 
-    for (int b0 = 0; b0 < nblk; b0 += kPrefetch) {
+    float *red = reinterpret_cast<float *>(bp + L.red);
+    if (!is_u) {
+        // ---- 64 weight rows: warp w owns rows 16w .. 16w+15
+        const int rg = 16 * warp + gid;  // and rg + 8 (same row mod 8)
+        const uint32_t zg = 128u + p.z[n0 + rg], zh = 128u + p.z[n0 + rg + 8];
+        const uint32_t nbg = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)zg));
+        const uint32_t nbh = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)zh));
+        const uint32_t negg = nbg | (nbg << 16), negh = nbh | (nbh << 16);
+        for (int c = 0; c < nch && ok; ++c) {
+            ok = wait_bounded(bar_chunk + 8 * c, 0);
+            const uint8_t *ctile = bp + L.codes + c * 8192;
 #pragma unroll
-        for (int i = 0; i < kPrefetch; ++i) {
-            const int b = b0 + i;
-            if (b < nblk) {
-                const uint4 cw = wg[i], hw = wh[i];
-                if (b + kPrefetch < nblk) {
-                    wg[i] = ld_stream(cg + 16 * (b + kPrefetch));
-                    wh[i] = ld_stream(ch + 16 * (b + kPrefetch));
+            for (int sb = 0; sb < 4; ++sb) {
+                // codes k = 64 sb + 16 cl + {0..15} of rows rg and rg + 8 (8 bytes each)
+                const int chunk = ((2 * sb + (cl >> 1)) ^ (rg & 7)) * 16 + (cl & 1) * 8;
+                const uint2 wgv = *reinterpret_cast<const uint2 *>(ctile + rg * 128 + chunk);
+                const uint2 whv = *reinterpret_cast<const uint2 *>(ctile + (rg + 8) * 128 + chunk);
+                const uint8_t *xt = bp + L.x + (4 * c + sb) * (TOK * 128);
+                uint4 xv[T][2];
+#pragma unroll
+                for (int n = 0; n < T; ++n) {
+                    const int t = 8 * n + gid;
+                    xv[n][0] = *reinterpret_cast<const uint4 *>(xt + t * 128 + (((2 * cl) ^ (t & 7)) << 4));
+                    xv[n][1] = *reinterpret_cast<const uint4 *>(xt + t * 128 + (((2 * cl + 1) ^ (t & 7)) << 4));
                 }
-                const uint32_t cgw[4] = {cw.x, cw.y, cw.z, cw.w};
-                const uint32_t chw[4] = {hw.x, hw.y, hw.z, hw.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    // codes k = 32c + 8j + {0..7}: pairs (0,4) (1,5) (2,6) (3,7)
-                    const uint32_t g0 = dequant_pair(cgw[j], negg), g1 = dequant_pair(cgw[j] >> 4, negg);
-                    const uint32_t g2 = dequant_pair(cgw[j] >> 8, negg), g3 = dequant_pair(cgw[j] >> 12, negg);
-                    const uint32_t h0 = dequant_pair(chw[j], negh), h1 = dequant_pair(chw[j] >> 4, negh);
-                    const uint32_t h2 = dequant_pair(chw[j] >> 8, negh), h3 = dequant_pair(chw[j] >> 12, negh);
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t wgw = j ? wgv.y : wgv.x, whw = j ? whv.y : whv.x;
+                    // codes k = 8j + {0..7}: pairs (0,4) (1,5) (2,6) (3,7)
+                    const uint32_t g0 = dequant_pair(wgw, negg), g1 = dequant_pair(wgw >> 4, negg);
+                    const uint32_t g2 = dequant_pair(wgw >> 8, negg), g3 = dequant_pair(wgw >> 12, negg);
+                    const uint32_t h0 = dequant_pair(whw, negh), h1 = dequant_pair(whw >> 4, negh);
+                    const uint32_t h2 = dequant_pair(whw >> 8, negh), h3 = dequant_pair(whw >> 12, negh);
 #pragma unroll
                     for (int n = 0; n < T; ++n) {
-                        const int t = 8 * n + gid;
-                        const uint4 xv = xs[(t * nblk + b) * 16 + swz(t, c, j)];
-                        const uint32_t b00 = prmt(xv.x, xv.z, 0x5410), b01 = prmt(xv.x, xv.z, 0x7632);
-                        const uint32_t b10 = prmt(xv.y, xv.w, 0x5410), b11 = prmt(xv.y, xv.w, 0x7632);
-                        mma_bf16_16816(acc[n], g0, h0, g1, h1, b00, b01);
-                        mma_bf16_16816(acc[n], g2, h2, g3, h3, b10, b11);
+                        const uint4 v = xv[n][j];
+                        mma_bf16_16816(acc[n], g0, h0, g1, h1, prmt(v.x, v.z, 0x5410), prmt(v.x, v.z, 0x7632));
+                        mma_bf16_16816(acc[n], g2, h2, g3, h3, prmt(v.y, v.w, 0x5410), prmt(v.y, v.w, 0x7632));
                     }
                 }
             }
         }
+#pragma unroll
+        for (int n = 0; n < T; ++n) {
+            const int col = 8 * n + 2 * cl;
+            red[rg * TOK + col] = acc[n][0];
+            red[rg * TOK + col + 1] = acc[n][1];
+            red[(rg + 8) * TOK + col] = acc[n][2];
+            red[(rg + 8) * TOK + col + 1] = acc[n][3];
+        }
+    } else {
+        // ---- 16 rows of G = [w_g; A^T]: warp w takes the 64-wide sub-tiles i = w (mod 4)
+        for (int i = warp; i < nsub && ok; i += 4) {
+            ok = wait_bounded(bar_chunk + 8 * (i >> 2), 0);
+            const uint8_t *gt = bp + L.codes + i * 2048;
+            const uint8_t *xt = bp + L.x + i * (TOK * 128);
+            const int ra = gid, rb = gid + 8;
+            const uint4 a0 = *reinterpret_cast<const uint4 *>(gt + ra * 128 + (((2 * cl) ^ (ra & 7)) << 4));
+            const uint4 a1 = *reinterpret_cast<const uint4 *>(gt + ra * 128 + (((2 * cl + 1) ^ (ra & 7)) << 4));
+            const uint4 b0 = *reinterpret_cast<const uint4 *>(gt + rb * 128 + (((2 * cl) ^ (rb & 7)) << 4));
+            const uint4 b1 = *reinterpret_cast<const uint4 *>(gt + rb * 128 + (((2 * cl + 1) ^ (rb & 7)) << 4));
+            const uint32_t ga[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const uint32_t ha[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int n = 0; n < T; ++n) {
+                const int t = 8 * n + gid;
+                const uint4 x0 = *reinterpret_cast<const uint4 *>(xt + t * 128 + (((2 * cl) ^ (t & 7)) << 4));
+                const uint4 x1 = *reinterpret_cast<const uint4 *>(xt + t * 128 + (((2 * cl + 1) ^ (t & 7)) << 4));
+                const uint32_t xa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                // natural pairs: step s covers k = 16 cl + 4s + {0,1} and + {2,3}
+#pragma unroll
+                for (int s = 0; s < 4; ++s)
+                    mma_bf16_16816(acc[n], ga[2 * s], ha[2 * s], ga[2 * s + 1], ha[2 * s + 1], xa[2 * s],
+                                   xa[2 * s + 1]);
+            }
+        }
+        float *mine = red + warp * 16 * TOK;  // [4 warps][16][TOK]
+#pragma unroll
+        for (int n = 0; n < T; ++n) {
+            const int col = 8 * n + 2 * cl;
+            mine[gid * TOK + col] = acc[n][0];
+            mine[gid * TOK + col + 1] = acc[n][1];
+            mine[(gid + 8) * TOK + col] = acc[n][2];
+            mine[(gid + 8) * TOK + col + 1] = acc[n][3];
+        }
+        __syncthreads();
+        for (int e = tid; e < 16 * TOK; e += 128)
+            red[e] = red[e] + red[16 * TOK + e] + red[32 * TOK + e] + red[48 * TOK + e];
+    }
+    if (!ok)
+        atomicOr(p.status, kStatusTimeout);
+    __syncthreads();
+    if (tid == 0) {
+        // no copy of this CTA may still be landing when it goes on (bounded;
+        // immediate unless a wait above gave up)
+        for (int c = 0; c < nch; ++c)
+            wait_bounded(bar_chunk + 8 * c, 0);
+        wait_bounded(bar_x, 0);
     }
 
-    // ---- partial tile [64 rows][TOK] to shared memory
-    __syncthreads();  // every warp is done reading xs
-    float *red = reinterpret_cast<float *>(smem_u4);
+    // ---- sum the K split over the cluster, in rank order, in the first CTA
+    __syncthreads();
+    cluster_sync();
+    const int tile = (is_u ? 16 : kRows) * TOK;
+    if (rank == 0) {
+        const uint32_t red_addr = base + L.red;
+        for (int e4 = tid; e4 < tile / 4; e4 += 128) {
+            // issue every remote load before summing (in rank order)
+            float4 o[8];
 #pragma unroll
-    for (int n = 0; n < T; ++n) {
-        const int r0 = warp * 16 + gid, col = 8 * n + 2 * c;
-        red[r0 * TOK + col] = acc[n][0];
-        red[r0 * TOK + col + 1] = acc[n][1];
-        red[(r0 + 8) * TOK + col] = acc[n][2];
-        red[(r0 + 8) * TOK + col + 1] = acc[n][3];
+            for (int q = 1; q < 8; ++q)
+                if (q < CS)
+                    o[q] = ld_dsmem_f4(map_to_rank(red_addr + 16 * e4, (uint32_t)q));
+            float4 s = reinterpret_cast<const float4 *>(red)[e4];
+#pragma unroll
+            for (int q = 1; q < 8; ++q)
+                if (q < CS) {
+                    s.x += o[q].x;
+                    s.y += o[q].y;
+                    s.z += o[q].z;
+                    s.w += o[q].w;
+                }
+            reinterpret_cast<float4 *>(red)[e4] = s;
+        }
     }
+    cluster_sync();  // the other CTAs' shared memory is no longer read
+    if (rank != 0)
+        return;
     __syncthreads();
 
-    constexpr int kTile = kRows * TOK;
-    if (p.S > 1) {
-        float *mine = p.part + ((size_t)nb * p.S + ks) * kTile;
-        for (int e = tid; e < kTile; e += 128)
-            mine[e] = red[e];
-        __threadfence();
-        __syncthreads();
-        if (tid == 0)
-            s_last = (atomicAdd(&p.counters[nb], 1u) == (unsigned)(p.S - 1));
-        __syncthreads();
-        if (!s_last)
-            return;
-        __threadfence();
-        const float *all = p.part + (size_t)nb * p.S * kTile;
-        for (int e = tid; e < kTile; e += 128) {
-            float sum = 0.f;
-            for (int q = 0; q < p.S; ++q)
-                sum += __ldcg(all + (size_t)q * kTile + e);
-            red[e] = sum;
+    if (is_u) {
+        // publish u rows 16*cluster .. +15 for all TOK token columns
+        for (int e = tid; e < 16 * TOK; e += 128) {
+            const int row = e / TOK, t = e - row * TOK;
+            p.ws_u[(16 * cluster + row) * kUStride + t] = red[e];
         }
+        __threadfence();
+        __syncthreads();
         if (tid == 0)
-            p.counters[nb] = 0u;
+            atomicAdd(&p.flags[0], 1u);
+        return;
+    }
+
+    // ---- epilogue of a 64-row cluster
+    float *us = reinterpret_cast<float *>(bp + L.u);   // u [R1p][TOK]
+    float *gs = us + p.R1p * TOK;                      // g [TOK]
+    float *vv = gs + TOK;                              // v [TOK][rp] = g * u
+    if (p.JB > 0) {
+        if (tid == 0) {
+            int good = 1;
+            const unsigned long long t0 = globaltimer();
+            while (ld_acquire_gpu(&p.flags[0]) < (unsigned)p.JB) {
+                if (globaltimer() - t0 > kWaitBudgetNs) {
+                    atomicOr(p.status, kStatusTimeout);
+                    good = 0;
+                    break;
+                }
+                __nanosleep(64);
+            }
+            s_ok = good;
+        }
+        __syncthreads();
+        for (int e = tid; e < p.R1p * TOK; e += 128) {
+            const int row = e / TOK, t = e - row * TOK;
+            us[e] = s_ok ? __ldcg(p.ws_u + row * kUStride + t) : 0.f;
+        }
+        __syncthreads();
+        if (tid == 0 && atomicAdd(&p.flags[1], 1u) == (unsigned)(p.NC - 1)) {
+            // every 64-row cluster has read u: reset for the next forward
+            p.flags[1] = 0u;
+            p.flags[0] = 0u;
+        }
+        if (tid < TOK)
+            gs[tid] = 1.0f / (1.0f + expf(-(us[tid] + p.b_g)));
+        __syncthreads();
+        for (int e = tid; e < TOK * p.rp; e += 128) {
+            const int t = e / p.rp, j = e - t * p.rp;
+            vv[e] = j < p.r ? gs[t] * us[(1 + j) * TOK + t] : 0.f;
+        }
         __syncthreads();
     }
 
-    // ---- epilogue: scale, EC up-projection, one rounding to bf16
-    const int row = tid & (kRows - 1), th = tid >> 6;  // two token phases
-    const int64_t n = (int64_t)nb * kRows + row;
-    const float sn = p.s[n];
+    const int row = tid & (kRows - 1), th = tid >> 6;
+    const int64_t n = n0 + row;
     float out[TOK / 2];
 #pragma unroll
     for (int i = 0; i < TOK / 2; ++i)
-        out[i] = sn * red[row * TOK + th + 2 * i];
-    if (p.ec) {
-        const uint16_t *bt = p.Bt + n * p.rp;
-        for (int j = 0; j < p.rp; j += 8) {
-            const uint4 bv = ld_nc(bt + j);
+        out[i] = s_epi * red[row * TOK + th + 2 * i];
+    if (p.JB > 0) {
+        // corr = sum_j v[t][j] * B^T[n][j]: B^T row in registers (8 values per 16 bytes),
+        // v broadcast from shared memory
+        const uint16_t *btg = p.Bt + n * p.rp;
+        auto accumulate = [&](int j0, const uint4 bv) {
             const float bj[8] = {bf16_lo(bv.x), bf16_hi(bv.x), bf16_lo(bv.y), bf16_hi(bv.y),
                                  bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
 #pragma unroll
             for (int i = 0; i < TOK / 2; ++i) {
-                const int t = th + 2 * i;
-                if (t < p.M) {
-                    const uint4 vv = __ldcg(reinterpret_cast<const uint4 *>(p.v + (int64_t)t * p.rp + j));
-                    out[i] += bf16_lo(vv.x) * bj[0] + bf16_hi(vv.x) * bj[1] + bf16_lo(vv.y) * bj[2] +
-                              bf16_hi(vv.y) * bj[3] + bf16_lo(vv.z) * bj[4] + bf16_hi(vv.z) * bj[5] +
-                              bf16_lo(vv.w) * bj[6] + bf16_hi(vv.w) * bj[7];
-                }
+                const float4 *vt = reinterpret_cast<const float4 *>(vv + (th + 2 * i) * p.rp + j0);
+                const float4 v0 = vt[0], v1 = vt[1];
+                out[i] += v0.x * bj[0] + v0.y * bj[1] + v0.z * bj[2] + v0.w * bj[3] + v1.x * bj[4] +
+                          v1.y * bj[5] + v1.z * bj[6] + v1.w * bj[7];
             }
-        }
-    }
-    if (n < p.N) {
+        };
 #pragma unroll
-        for (int i = 0; i < TOK / 2; ++i) {
-            const int t = th + 2 * i;
-            if (t < p.M)
-                p.y[(int64_t)t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
-        }
+        for (int q = 0; q < 8; ++q)
+            if (8 * q < p.rp)
+                accumulate(8 * q, bt_pre[q]);
+        for (int j0 = 64; j0 < p.rp; j0 += 8)
+            accumulate(j0, ld_nc(btg + j0));
+    }
+#pragma unroll
+    for (int i = 0; i < TOK / 2; ++i) {
+        const int t = th + 2 * i;
+        if (t < p.M && n < p.N)
+            p.y[(int64_t)t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
     }
 }
 
-void pick_split(const Packed &pk, int num_sms, int &S, int &bps)
+// Cluster size CS (CTAs splitting K) and the k per CTA, or 0 if a slice would
+// not fit in shared memory.  Up to 8 CTAs per cluster, fewer when the grid
+// would exceed about 8 CTAs per SM.
+int pick_cluster(const Packed &pk, int num_sms, int JB, int *KS_out)
 {
-    const int nkb = (int)(pk.Kp / 128);
-    const int nblocks = (int)(pk.Np / kRows);
-    // aim for about four CTAs per SM, at most kMaxBps k blocks per CTA
-    int target = std::max(1, (4 * num_sms + nblocks - 1) / nblocks);
-    S = std::min(target, nkb);
-    bps = (nkb + S - 1) / S;
-    if (bps > kMaxBps)
-        bps = kMaxBps;
-    S = (nkb + bps - 1) / bps;
+    const int NC = (int)(pk.Np / kRows);
+    const int chunks = (int)(pk.Kp / kChunk);
+    int CS = std::min(8, chunks);
+    // no more than about 8 CTAs per SM, and no rank left without a chunk
+    while (CS > 1 && ((int64_t)(NC + JB) * CS > 8LL * num_sms || (CS - 1) * ((chunks + CS - 1) / CS) >= chunks))
+        --CS;
+    const int per = (chunks + CS - 1) / CS;
+    if (per > kMaxChunks)
+        return 0;
+    *KS_out = per * kChunk;
+    return CS;
+}
+
+template <int T>
+const void *kernel_ptr()
+{
+    return reinterpret_cast<const void *>(decode_w4ec_kernel<T>);
 }
 
 }  // namespace
 
-size_t decode_part_floats(const Packed &pk, int num_sms)
+bool decode_supported(const Packed &pk, int num_sms)
 {
-    int S, bps;
-    pick_split(pk, num_sms, S, bps);
-    return S > 1 ? (size_t)(pk.Np / kRows) * S * kRows * kDecodeMaxTokens : 0;
+    if (pk.rp > 128)
+        return false;
+    int KS = 0;
+    const int CS = pick_cluster(pk, num_sms, pk.r > 0 ? pk.R1p / 16 : 0, &KS);
+    if (CS == 0)
+        return false;
+    return smem_layout<32>(KS, pk.rp, pk.R1p).total + 1024 <= 227 * 1024;
 }
 
-int decode_counters(const Packed &pk) { return (int)(pk.Np / kRows); }
+cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
+{
+    Maps *m = static_cast<Maps *>(w.maps);
+    if (!m) {
+        m = new (std::nothrow) Maps();
+        if (!m)
+            return cudaErrorMemoryAllocation;
+        w.maps = m;
+    }
+    cudaError_t e = make_map(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)pk.Kp / 8,
+                             (uint64_t)pk.Np, 32, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess && pk.r > 0)
+        e = make_map(&m->g, pk.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.Kp, (uint64_t)pk.R1p, 64, 16,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess && pk.r > 0)
+        e = make_map(&m->bt, pk.Bt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.rp, (uint64_t)pk.Np,
+                     (uint32_t)pk.rp, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e == cudaSuccess && pk.r == 0) {
+        m->g = m->codes;
+        m->bt = m->codes;
+    }
+    return e;
+}
 
-cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, const uint16_t *v,
-                          bool ec, const DecodeWork &w, cudaStream_t st,
-                          int num_sms)
+void decode_free(DecodeWork &w)
+{
+    delete static_cast<Maps *>(w.maps);
+    w.maps = nullptr;
+}
+
+size_t decode_u_floats(const Packed &pk) { return (size_t)pk.R1p * kUStride; }
+
+cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, bool ec, const DecodeWork &w,
+                          int *status, cudaStream_t st, int num_sms)
 {
     if (M <= 0)
         return cudaSuccess;
-    if (M > kDecodeMaxTokens)
+    if (M > kDecodeMaxTokens || !w.maps)
         return cudaErrorInvalidValue;
+    const Maps *m = static_cast<const Maps *>(w.maps);
+    const bool use_ec = ec && pk.r > 0;
     DecodeParams p;
-    p.codes = pk.codes;
+    p.Bt = pk.Bt;
     p.s = pk.s;
     p.z = pk.z;
-    p.x = static_cast<const uint16_t *>(x);
     p.y = static_cast<uint16_t *>(y);
-    p.v = v;
-    p.Bt = pk.Bt;
-    p.part = w.part;
-    p.counters = w.counters;
+    p.ws_u = w.ws_u;
+    p.flags = w.flags;
+    p.status = status;
     p.M = M;
-    p.K = pk.K;
-    p.Kp = pk.Kp;
     p.N = pk.N;
-    p.rp = pk.rp;
-    p.ec = (ec && pk.r > 0) ? 1 : 0;
-    pick_split(pk, num_sms, p.S, p.bps);
-    const int T = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
-    const int nblocks = (int)(pk.Np / kRows);
-    if (nblocks > w.n_counters || (p.S > 1 && (size_t)nblocks * p.S * kRows * 8 * T > w.part_floats))
+    p.JB = use_ec ? pk.R1p / 16 : 0;
+    p.NC = (int)(pk.Np / kRows);
+    int KS = 0;
+    const int CS = pick_cluster(pk, num_sms, p.JB, &KS);
+    if (CS == 0)
         return cudaErrorInvalidValue;
-    const size_t smem = std::max((size_t)8 * T * p.bps * 256, (size_t)kRows * 8 * T * sizeof(float));
+    p.Kp = pk.Kp;
+    p.KS = KS;
+    p.nch = KS / kChunk;
+    p.r = pk.r;
+    p.rp = use_ec ? pk.rp : 0;
+    p.R1p = use_ec ? pk.R1p : 0;
+    p.b_g = pk.b_g;
+    const int T = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
+    CUtensorMap tm_x;
+    cudaError_t e = make_map(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.K, (uint64_t)M, 64,
+                             (uint32_t)(8 * T), CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess)
+        return e;
+    const Smem L = T == 1 ? smem_layout<8>(p.KS, p.rp, p.R1p)
+                          : (T == 2 ? smem_layout<16>(p.KS, p.rp, p.R1p) : smem_layout<32>(p.KS, p.rp, p.R1p));
+    const size_t smem = L.total + 1024;
+    const void *fn = T == 1 ? kernel_ptr<1>() : (T == 2 ? kernel_ptr<2>() : kernel_ptr<4>());
+    e = raise_smem_limit(fn, smem);
+    if (e != cudaSuccess)
+        return e;
 
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(nblocks * p.S));
+    cfg.gridDim = dim3((unsigned)((p.JB + p.NC) * CS));
     cfg.blockDim = dim3(128);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = CS;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    void (*fn)(DecodeParams) = T == 1 ? decode_w4ec_kernel<1> : (T == 2 ? decode_w4ec_kernel<2> : decode_w4ec_kernel<4>);
-    if (smem > 48 * 1024) {
-        cudaError_t e = raise_smem_limit(reinterpret_cast<const void *>(fn), smem);
-        if (e != cudaSuccess)
-            return e;
+    cfg.numAttrs = 2;
+    switch (T) {
+    case 1: return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<1>, m->codes, m->g, m->bt, tm_x, p, CS);
+    case 2: return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<2>, m->codes, m->g, m->bt, tm_x, p, CS);
+    default: return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<4>, m->codes, m->g, m->bt, tm_x, p, CS);
     }
-    return cudaLaunchKernelEx(&cfg, fn, p);
 }
 
 }  // namespace spear

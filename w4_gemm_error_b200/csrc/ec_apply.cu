@@ -3,7 +3,7 @@
 // kernel-fusion dispatch (SPEAR, "A System for Post-Quantization
 // Error-Adaptive Recovery Enabling Efficient Low-Bit LLM Serving", Abstract)
 // weighs against the fused kernels; y is rounded to bf16 twice on this path
-// (after the GEMM and after the correction).
+// (after the GEMM and after the correction); v is read in fp32.
 //
 // One thread per output channel n (consecutive n -> coalesced y rows), a CTA
 // handles 256 channels and 32 tokens; v for those tokens is staged in shared
@@ -18,7 +18,7 @@ constexpr int kThreads = 256;
 constexpr int kTokChunk = 32;
 
 __global__ void __launch_bounds__(kThreads)
-ec_apply_kernel(const uint16_t *__restrict__ v, const uint16_t *__restrict__ Bt, uint16_t *__restrict__ y,
+ec_apply_kernel(const float *__restrict__ vf, const uint16_t *__restrict__ Bt, uint16_t *__restrict__ y,
                 int64_t M, int64_t N, int rp)
 {
     extern __shared__ float vs[];  // [kTokChunk][rp]
@@ -28,7 +28,7 @@ ec_apply_kernel(const uint16_t *__restrict__ v, const uint16_t *__restrict__ Bt,
     const int ntok = (int)min((int64_t)kTokChunk, M - t0);
     for (int e = threadIdx.x; e < kTokChunk * rp; e += kThreads) {
         const int tt = e / rp, j = e - tt * rp;
-        vs[e] = tt < ntok ? __uint_as_float((uint32_t)v[(t0 + tt) * rp + j] << 16) : 0.f;
+        vs[e] = tt < ntok ? vf[(t0 + tt) * rp + j] : 0.f;
     }
     __syncthreads();
     const int64_t n = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -62,7 +62,7 @@ ec_apply_kernel(const uint16_t *__restrict__ v, const uint16_t *__restrict__ Bt,
 
 }  // namespace
 
-cudaError_t launch_ec_apply(const Packed &pk, const uint16_t *v, void *y, int64_t M, cudaStream_t st)
+cudaError_t launch_ec_apply(const Packed &pk, const float *vf, void *y, int64_t M, cudaStream_t st)
 {
     if (M <= 0 || pk.r == 0)
         return cudaSuccess;
@@ -83,7 +83,7 @@ cudaError_t launch_ec_apply(const Packed &pk, const uint16_t *v, void *y, int64_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ec_apply_kernel, v, (const uint16_t *)pk.Bt, static_cast<uint16_t *>(y), M,
+    return cudaLaunchKernelEx(&cfg, ec_apply_kernel, vf, (const uint16_t *)pk.Bt, static_cast<uint16_t *>(y), M,
                               pk.N, pk.rp);
 }
 

@@ -16,7 +16,10 @@ cudaError_t raise_smem_limit(const void *func, size_t bytes);
 //   z     [Np] uint8          per-channel zero point (8)
 //   G     [R1p][Kp] bf16      row 0 = w_g, rows 1..r = A^T, other rows 0
 //   Bt    [Np][rp] bf16       B transposed (Bt[n][j] = B[j][n]), zero padded
-// Np = N rounded up to 128, Kp = K rounded up to 128, rp = r rounded up to 16,
+//   Bts   [Np][rp] bf16       Bt[n][j] / e[n] with e[n] = s[n] (1 where s[n] = 0): the EC
+//                             operand of kernels that accumulate sum_k x (q - z) unscaled
+//                             and apply e[n] once at the end
+// Np = N rounded up to 128, Kp = K rounded up to 256, rp = r rounded up to 16,
 // R1p = (r + 1) rounded up to 16.
 struct Packed {
     int64_t K, N, Kp, Np;
@@ -26,6 +29,7 @@ struct Packed {
     uint8_t *z;
     uint16_t *G;
     uint16_t *Bt;
+    uint16_t *Bts;
     float b_g;
 };
 
@@ -45,26 +49,29 @@ struct PrepassWork {
     unsigned *counters;   // one per 16-token tile, zero between calls
     int n_counters;
 };
-cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t *v, float *g,
+// vf (may be null) receives v in fp32 [M][rp] for kernels that do not need a bf16 operand.
+cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t *v, float *vf, float *g,
                            const PrepassWork &w, cudaStream_t st, int num_sms);
 size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms);
 int prepass_counters(int64_t max_M);
 
-// ---- decode main kernel: tensor-core (mma.sync) split-K W4 GEMM, tokens on
-// the narrow side, EC applied in the epilogue when `ec` is set.
+// ---- decode kernel: clusters of CTAs split K over 64 weight rows, mma.sync
+// on exact int4 codes, EC down-projection on extra clusters of the same grid
+// and EC up-projection in the epilogue (when `ec` is set).
 struct DecodeWork {
-    float *part;
-    size_t part_floats;
-    unsigned *counters;   // one per 64-row block, zero between calls
-    int n_counters;
+    void *maps;           // tensor maps of the packed operands (host memory)
+    float *ws_u;          // [R1p][32] published EC down-projection
+    unsigned *flags;      // two counters, zero between calls
 };
 constexpr int kDecodeMaxTokens = 32;   // tokens per launch
-cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, const uint16_t *v,
-                          bool ec, const DecodeWork &w, cudaStream_t st, int num_sms);
-size_t decode_part_floats(const Packed &pk, int num_sms);
-int decode_counters(const Packed &pk);
+bool decode_supported(const Packed &pk, int num_sms);
+cudaError_t decode_prepare(const Packed &pk, DecodeWork &w);
+void decode_free(DecodeWork &w);
+size_t decode_u_floats(const Packed &pk);
+cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, bool ec, const DecodeWork &w,
+                          int *status, cudaStream_t st, int num_sms);
 
-// ---- split EC: y[t][n] = bf16(y[t][n] + sum_j v[t][j] * Bt[n][j])
-cudaError_t launch_ec_apply(const Packed &pk, const uint16_t *v, void *y, int64_t M, cudaStream_t st);
+// ---- split EC: y[t][n] = bf16(y[t][n] + sum_j v[t][j] * Bt[n][j]), v in fp32
+cudaError_t launch_ec_apply(const Packed &pk, const float *vf, void *y, int64_t M, cudaStream_t st);
 
 }  // namespace spear

@@ -82,10 +82,12 @@ pack_w4_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K, int64_t Np,
 }
 
 // G [R1p][Kp]: row 0 = w_g, rows 1..r = A^T;  Bt [Np][rp] = B^T; zeros elsewhere.
+// Bts = Bt / e[n], e[n] = s[n] (1 where s[n] = 0), in fp32 rounded once to bf16.
 __global__ void pack_ec_kernel(const uint16_t *__restrict__ A, const uint16_t *__restrict__ B,
-                               const uint16_t *__restrict__ wg, int64_t K, int64_t N, int r,
-                               int64_t Kp, int64_t Np, int R1p, int rp, uint16_t *__restrict__ G,
-                               uint16_t *__restrict__ Bt)
+                               const uint16_t *__restrict__ wg, const float *__restrict__ s, int64_t K,
+                               int64_t N, int r, int64_t Kp, int64_t Np, int R1p, int rp,
+                               uint16_t *__restrict__ G, uint16_t *__restrict__ Bt, uint16_t *__restrict__ Bts,
+                               int *status)
 {
     const int64_t nG = (int64_t)R1p * Kp, nB = Np * rp;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nG + nB;
@@ -102,7 +104,14 @@ __global__ void pack_ec_kernel(const uint16_t *__restrict__ A, const uint16_t *_
             G[i] = v;
         } else {
             const int64_t e = i - nG, n = e / rp, j = e - n * rp;
-            Bt[e] = (n < N && j < r) ? B[j * N + n] : (uint16_t)0;
+            const uint16_t b = (n < N && j < r) ? B[j * N + n] : (uint16_t)0;
+            Bt[e] = b;
+            const float sn = s[n];
+            const float q = __fdiv_rn(__uint_as_float((uint32_t)b << 16), sn != 0.0f ? sn : 1.0f);
+            const __nv_bfloat16 qb = __float2bfloat16_rn(q);
+            if (!isfinite(__bfloat162float(qb)))
+                atomicOr(status, kStatusNonFinite);
+            Bts[e] = __bfloat16_as_ushort(qb);
         }
     }
 }
@@ -119,8 +128,8 @@ cudaError_t launch_pack(const Packed &pk, const void *W, const void *A, const vo
     if (e != cudaSuccess || pk.r == 0)
         return e;
     pack_ec_kernel<<<1024, 256, 0, st>>>(static_cast<const uint16_t *>(A), static_cast<const uint16_t *>(B),
-                                         static_cast<const uint16_t *>(wg), pk.K, pk.N, pk.r, pk.Kp, pk.Np,
-                                         pk.R1p, pk.rp, pk.G, pk.Bt);
+                                         static_cast<const uint16_t *>(wg), pk.s, pk.K, pk.N, pk.r, pk.Kp,
+                                         pk.Np, pk.R1p, pk.rp, pk.G, pk.Bt, pk.Bts, status);
     return cudaGetLastError();
 }
 

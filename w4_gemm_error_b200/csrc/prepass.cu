@@ -33,6 +33,7 @@ struct PrepassParams {
     int S;       // CTAs per token tile (split-K)
     int bps;     // 64-wide k blocks per split
     uint16_t *v;
+    float *vf;
     float *g;
     float *part;
     unsigned *counters;
@@ -153,6 +154,8 @@ __global__ void __launch_bounds__(128) prepass_kernel(PrepassParams p)
             continue;
         const float val = (j < p.r) ? s_gate[tt] * red[(1 + j) * kTok + tt] : 0.f;
         p.v[t * p.rp + j] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
+        if (p.vf)
+            p.vf[t * p.rp + j] = val;
     }
 }
 
@@ -201,7 +204,7 @@ size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms)
 
 int prepass_counters(int64_t max_M) { return (int)((max_M + kTok - 1) / kTok); }
 
-cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t *v, float *g,
+cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t *v, float *vf, float *g,
                            const PrepassWork &w, cudaStream_t st, int num_sms)
 {
     if (M <= 0 || pk.r == 0)
@@ -221,6 +224,7 @@ cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t 
     p.bps = (nkb + p.S - 1) / p.S;
     p.S = (nkb + p.bps - 1) / p.bps;  // drop empty splits
     p.v = v;
+    p.vf = vf;
     p.g = g;
     p.part = w.part;
     p.counters = w.counters;

@@ -11,7 +11,7 @@
 #include <new>
 #include <vector>
 
-#include "../../include/spear_w4ec.h"
+#include "spear_w4ec.h"
 #include "device_utils.cuh"
 #include "kernels.h"
 #include "tc_gemm.h"
@@ -26,6 +26,7 @@ struct spear_w4ec {
     bool packed = false;
     // workspace
     uint16_t *v = nullptr;      // [max_M][rp] bf16: g_t * (x . A)
+    float *vf = nullptr;        // the same in fp32 (split path)
     float *gbuf = nullptr;      // [max_M] gate values
     PrepassWork pre{};
     DecodeWork dec{};
@@ -105,12 +106,15 @@ void free_all(spear_w4ec *h)
     cudaFree(h->pk.z);
     cudaFree(h->pk.G);
     cudaFree(h->pk.Bt);
+    cudaFree(h->pk.Bts);
     cudaFree(h->v);
+    cudaFree(h->vf);
     cudaFree(h->gbuf);
     cudaFree(h->pre.part);
     cudaFree(h->pre.counters);
-    cudaFree(h->dec.part);
-    cudaFree(h->dec.counters);
+    cudaFree(h->dec.ws_u);
+    cudaFree(h->dec.flags);
+    decode_free(h->dec);
     tc_free(h->tc);
     cudaFree(h->status);
     cudaFree(h->x_stage);
@@ -138,7 +142,9 @@ uint32_t resolve(const spear_w4ec *h, int64_t M, uint32_t flags)
     const uint32_t tuned = h->table[bucket_of(M)];
     if (!path)
         path = tuned ? (tuned & (SPEAR_FORCE_DECODE | SPEAR_FORCE_TC))
-                     : ((M <= kDecodeMaxTokens || !tc_supported(h)) ? SPEAR_FORCE_DECODE : SPEAR_FORCE_TC);
+                     : (((M <= kDecodeMaxTokens && decode_supported(h->pk, h->num_sms)) || !tc_supported(h))
+                            ? SPEAR_FORCE_DECODE
+                            : SPEAR_FORCE_TC);
     if (!mode)
         mode = tuned ? (tuned & (SPEAR_FORCE_FUSED | SPEAR_FORCE_SPLIT)) : SPEAR_FORCE_FUSED;
     if (!mode)
@@ -159,8 +165,12 @@ int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t
     if (h->fault_launch)
         return SPEAR_ERR_CUDA;
     cudaError_t e = cudaSuccess;
-    if (ec) {
-        e = launch_prepass(pk, x, M, h->v, h->gbuf, h->pre, st, h->num_sms);
+    const bool decode = (choice & SPEAR_FORCE_DECODE) != 0;
+    if (decode && !decode_supported(pk, h->num_sms))
+        return SPEAR_ERR_UNSUPPORTED;
+    // the decode kernel computes its own gate and EC down-projection when fused
+    if (ec && !(decode && fused)) {
+        e = launch_prepass(pk, x, M, h->v, fused ? nullptr : h->vf, h->gbuf, h->pre, st, h->num_sms);
         if (e != cudaSuccess)
             return from_cuda(e);
     }
@@ -174,14 +184,14 @@ int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t
         for (int64_t t0 = 0; t0 < M; t0 += kDecodeMaxTokens) {
             const int64_t m = std::min<int64_t>(kDecodeMaxTokens, M - t0);
             e = launch_decode(pk, static_cast<const uint16_t *>(x) + t0 * pk.K,
-                              static_cast<uint16_t *>(y) + t0 * pk.N, m, h->v + t0 * pk.rp, ec && fused,
-                              h->dec, st, h->num_sms);
+                              static_cast<uint16_t *>(y) + t0 * pk.N, m, ec && fused, h->dec, h->status, st,
+                              h->num_sms);
             if (e != cudaSuccess)
                 return from_cuda(e);
         }
     }
     if (ec && !fused) {
-        e = launch_ec_apply(pk, h->v, y, M, st);
+        e = launch_ec_apply(pk, h->vf, y, M, st);
         if (e != cudaSuccess)
             return from_cuda(e);
     }
@@ -201,7 +211,7 @@ const char *spear_w4ec_strerror(int status)
     case SPEAR_ERR_NOMEM: return "out of memory";
     case SPEAR_ERR_CUDA: return "CUDA error";
     case SPEAR_ERR_TIMEOUT: return "device-side wait timed out";
-    case SPEAR_ERR_DEVICE: return "kernel reported bad data (non-finite weights)";
+    case SPEAR_ERR_DEVICE: return "kernel reported bad data (non-finite weights or scaled EC operand)";
     case SPEAR_ERR_STATE: return "call out of order (layer not packed)";
     default: return "unknown status";
     }
@@ -238,7 +248,7 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r, const s
     Packed &pk = h->pk;
     pk.K = K;
     pk.N = N;
-    pk.Kp = round_up(K, 128);
+    pk.Kp = round_up(K, 256);
     pk.Np = round_up(N, 128);
     pk.r = r;
     pk.rp = r > 0 ? (int)round_up(r, 16) : 0;
@@ -256,17 +266,17 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r, const s
     if (r > 0) {
         chk(alloc_zero(&pk.G, (size_t)pk.R1p * pk.Kp));
         chk(alloc_zero(&pk.Bt, (size_t)pk.Np * pk.rp));
+        chk(alloc_zero(&pk.Bts, (size_t)pk.Np * pk.rp));
         chk(alloc_zero(&h->v, (size_t)h->max_M * pk.rp));
+        chk(alloc_zero(&h->vf, (size_t)h->max_M * pk.rp));
         chk(alloc_zero(&h->gbuf, (size_t)h->max_M));
         h->pre.part_floats = prepass_part_floats(pk, h->max_M, h->num_sms);
         h->pre.n_counters = prepass_counters(h->max_M);
         chk(alloc_zero(&h->pre.part, h->pre.part_floats));
         chk(alloc_zero(&h->pre.counters, (size_t)h->pre.n_counters));
     }
-    h->dec.part_floats = decode_part_floats(pk, h->num_sms);
-    h->dec.n_counters = decode_counters(pk);
-    chk(alloc_zero(&h->dec.part, h->dec.part_floats));
-    chk(alloc_zero(&h->dec.counters, (size_t)h->dec.n_counters));
+    chk(alloc_zero(&h->dec.ws_u, decode_u_floats(pk)));
+    chk(alloc_zero(&h->dec.flags, (size_t)2));
     chk(tc_alloc(pk, h->max_M, h->num_sms, h->tc));
     chk(alloc_zero(&h->status, 1));
     if (e == cudaSuccess)
@@ -295,6 +305,8 @@ int spear_w4ec_pack(spear_w4ec *h, const void *W, const void *A, const void *B, 
     if (e != cudaSuccess)
         return from_cuda(e);
     e = tc_prepare(h->pk, h->tc);
+    if (e == cudaSuccess)
+        e = decode_prepare(h->pk, h->dec);
     if (e != cudaSuccess)
         return from_cuda(e);
     h->packed = true;
@@ -401,7 +413,7 @@ int spear_w4ec_get_gate(const spear_w4ec *h, const void *x, float *g, int64_t M,
         return SPEAR_OK;
     DeviceGuard guard(h->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_prepass(h->pk, x, M, h->v, h->gbuf, h->pre, st, h->num_sms);
+    cudaError_t e = launch_prepass(h->pk, x, M, h->v, nullptr, h->gbuf, h->pre, st, h->num_sms);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(g, h->gbuf, (size_t)M * sizeof(float), cudaMemcpyDeviceToDevice, st);
     return from_cuda(e);
@@ -450,6 +462,8 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
     const uint32_t paths[2] = {SPEAR_FORCE_DECODE, SPEAR_FORCE_TC};
     for (uint32_t path : paths) {
         if (path == SPEAR_FORCE_TC && !tc_supported(h))
+            continue;
+        if (path == SPEAR_FORCE_DECODE && !decode_supported(h->pk, h->num_sms))
             continue;
         cands.push_back(path | SPEAR_FORCE_FUSED);
         if (h->pk.r > 0)

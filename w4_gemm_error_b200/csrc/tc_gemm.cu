@@ -1,16 +1,363 @@
-// Placeholder until the tcgen05 tile kernel lands: reports the path as unavailable.
+// W4 GEMM with the Error Compensator as a second accumulation, on the
+// Blackwell tensor cores (tcgen05, accumulators in tensor memory, operands
+// staged by TMA).
+//
+// SPEAR, "A System for Post-Quantization Error-Adaptive Recovery Enabling
+// Efficient Low-Bit LLM Serving", Abstract: the post-EC computation is fused
+// into the low-bit GEMM.  Here the EC is literally part of the same
+// accumulation: after the K loop of the main product the tile runs r/16 more
+// MMA k-steps with v = g * (x . A) (from the prepass) against B^T, into the
+// same TMEM accumulator, so
+//     D[n, t] = sum_k (q[n,k] - z[n]) x[t,k] + sum_j (B[j,n] / s[n]) v[t,j]
+// and the epilogue writes y[t, n] = bf16(s[n] * D[n, t]).
+//
+// Layout of one CTA (persistent, one per SM, 10 warps):
+//   warp 0      TMA producer: x tile (256 tokens x 64 k, 128B-swizzled) and
+//               the int4 code tile (128 rows x 64 k) per stage; for the EC
+//               stages the B^T tile and the v tile instead.
+//   warp 1      TMEM allocator and the single MMA-issuing thread:
+//               tcgen05.mma.cta_group::1.kind::f16, M = 128 weight rows,
+//               N = 256 tokens, K = 16 per instruction (swap-AB: weights
+//               on the M side so one dequantised tile serves 256 tokens).
+//   warps 2-5   dequantisers: thread i owns weight row i of the tile and
+//               writes the exact integers (q - z) as bf16 into the
+//               128B-swizzled K-major A tile of the stage (the layout the
+//               MMA descriptor names).
+//   warps 6-9   epilogue: tcgen05.ld of the finished accumulator (each warp
+//               its 32-lane quarter), times the channel scale s[n], bf16
+//               rounding, stores of y[t, n].
+// The accumulator holds sum_k x (q - z) exactly up to fp32 summation, so the
+// EC stages use B^T / s[n] (prepared at pack time) and one multiplication by
+// s[n] in the epilogue scales both terms.
+// Four stages of 52 KB in shared memory; two 256-column accumulators in
+// TMEM so the epilogue of one tile overlaps the main loop of the next.
+// Every mbarrier wait is bounded (about a second of %globaltimer); a wait
+// that runs out sets the handle's status word and the kernel winds down.
+#include <new>
+
+#include "async_utils.cuh"
 #include "tc_gemm.h"
+#include "tensor_map.h"
 
 namespace spear {
+namespace {
 
-bool tc_available(const Packed &) { return false; }
-cudaError_t tc_alloc(const Packed &, int64_t, int, TcWork &) { return cudaSuccess; }
-void tc_free(TcWork &) {}
-cudaError_t tc_prepare(const Packed &, TcWork &) { return cudaSuccess; }
-cudaError_t launch_tc(const Packed &, const void *, void *, int64_t, const uint16_t *, bool, const TcWork &, int *,
-                      bool, cudaStream_t, int)
+constexpr int BM = 128;                       // weight rows per tile (TMEM lanes)
+constexpr int BN = 256;                       // tokens per tile (MMA N)
+constexpr int BK = 64;                        // k per stage: one 128-byte swizzle atom of bf16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;          // 16 KB dequantised weights (or B^T on EC stages)
+constexpr int B_BYTES = BN * BK * 2;          // 32 KB activations (or v on EC stages)
+constexpr int C_BYTES = BM * BK / 2;          // 4 KB int4 codes
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
+constexpr int THREADS = 320;
+constexpr int TMEM_COLS = 2 * BN;
+
+struct TcParams {
+    int64_t M, N;
+    int n_main, n_ec, rp;
+    int n_ttiles, n_tiles;
+    const float *s;
+    const uint8_t *z;
+    uint16_t *y;
+    int *status;
+};
+
+struct Maps {
+    CUtensorMap codes;
+    CUtensorMap bt;
+};
+
+// ---------------------------------------------------------------- the kernel
+
+__global__ void __launch_bounds__(THREADS, 1)
+tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
+               const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_v, TcParams p)
 {
-    return cudaErrorNotSupported;
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[3 * STAGES + 5];
+    __shared__ uint32_t tmem_base_slot;
+    __shared__ volatile int abort_flag;
+
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+    uint8_t *const base_ptr = smem_raw + (base - smem_addr(smem_raw));
+    const uint32_t full0 = smem_addr(&bars[0]);
+    const uint32_t aready0 = smem_addr(&bars[STAGES]);
+    const uint32_t empty0 = smem_addr(&bars[2 * STAGES]);
+    const uint32_t tfull0 = smem_addr(&bars[3 * STAGES]);
+    const uint32_t tempty0 = smem_addr(&bars[3 * STAGES + 2]);
+    const uint32_t drain = smem_addr(&bars[3 * STAGES + 4]);
+
+    if (tid == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(aready0 + 8 * s, 128);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(tfull0 + 8 * b, 1);
+            mbar_init(tempty0 + 8 * b, 128);
+        }
+        mbar_init(drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&tmem_base_slot)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_slot;
+    const int n_stages = p.n_main + p.n_ec;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            pdl_wait();  // x and v come from earlier kernels in the stream
+            uint32_t g = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+                const int t0 = (tile % p.n_ttiles) * BN, n0 = (tile / p.n_ttiles) * BM;
+                for (int st = 0; st < n_stages; ++st, ++g) {
+                    const uint32_t slot = g % STAGES, phase = (g / STAGES) & 1;
+                    if (!mbar_wait(empty0 + 8 * slot, phase ^ 1, &abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sb = base + slot * STAGE_BYTES;
+                    const uint32_t full = full0 + 8 * slot;
+                    if (st < p.n_main) {
+                        mbar_expect_tx(full, B_BYTES + C_BYTES);
+                        tma_load_2d(sb + A_BYTES, &tm_x, st * BK, t0, full);
+                        tma_load_2d(sb + A_BYTES + B_BYTES, &tm_codes, st * (BK / 8), n0, full);
+                    } else {
+                        const int e = st - p.n_main;
+                        mbar_expect_tx(full, A_BYTES + B_BYTES);
+                        tma_load_2d(sb, &tm_bt, e * BK, n0, full);
+                        tma_load_2d(sb + A_BYTES, &tm_v, e * BK, t0, full);
+                    }
+                }
+            }
+            // do not leave while copies this CTA issued may still land
+            for (uint32_t k = 0; k < STAGES && k < g; ++k) {
+                const uint32_t gg = g - 1 - k, slot = gg % STAGES, phase = (gg / STAGES) & 1;
+                mbar_wait_final(full0 + 8 * slot, phase);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = (1u << 4)                    // D: f32
+                                   | (1u << 7) | (1u << 10)     // A, B: bf16
+                                   | ((uint32_t)(BN >> 3) << 17)
+                                   | ((uint32_t)(BM >> 4) << 24);
+            uint32_t g = 0;
+            int lt = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++lt) {
+                const uint32_t buf = lt & 1;
+                if (!mbar_wait(tempty0 + 8 * buf, ((lt >> 1) & 1) ^ 1, &abort_flag, p.status))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + buf * BN;
+                for (int st = 0; st < n_stages; ++st, ++g) {
+                    const uint32_t slot = g % STAGES, phase = (g / STAGES) & 1;
+                    if (!mbar_wait(full0 + 8 * slot, phase, &abort_flag, p.status) ||
+                        !mbar_wait(aready0 + 8 * slot, phase, &abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sb = base + slot * STAGE_BYTES;
+                    const uint64_t a_desc = smem_desc_sw128(sb), b_desc = smem_desc_sw128(sb + A_BYTES);
+                    int ksteps = BK / 16;
+                    if (st >= p.n_main) {
+                        const int rem = p.rp - (st - p.n_main) * BK;
+                        ksteps = (rem < BK ? rem : BK) / 16;
+                    }
+                    for (int k = 0; k < ksteps; ++k)
+                        mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (st > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(empty0 + 8 * slot);
+                }
+                if (ok)
+                    mma_commit(tfull0 + 8 * buf);
+            }
+            // every MMA this thread issued is complete before TMEM is released
+            mma_commit(drain);
+            mbar_wait_final(drain, 0);
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------ dequantisers: thread i = weight row i
+        const int i = tid - 64;
+        uint32_t g = 0;
+        for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
+            const int n = (tile / p.n_ttiles) * BM + i;
+            const uint32_t zb = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + p.z[n])));
+            const uint32_t negz = zb | (zb << 16);
+            bool ok = true;
+            for (int st = 0; st < n_stages; ++st, ++g) {
+                const uint32_t slot = g % STAGES, phase = (g / STAGES) & 1;
+                if (!mbar_wait(full0 + 8 * slot, phase, &abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                if (st < p.n_main) {
+                    uint8_t *sb = base_ptr + slot * STAGE_BYTES;
+                    const uint4 *cw = reinterpret_cast<const uint4 *>(sb + A_BYTES + B_BYTES + i * 32);
+                    const uint4 w0 = cw[0], w1 = cw[1];
+                    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    uint8_t *arow = sb + i * 128;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        // codes k = 8j + {0..7}: pairs (0,4) (1,5) (2,6) (3,7)
+                        const uint32_t p0 = dequant_pair(words[j], negz), p1 = dequant_pair(words[j] >> 4, negz);
+                        const uint32_t p2 = dequant_pair(words[j] >> 8, negz), p3 = dequant_pair(words[j] >> 12, negz);
+                        uint4 o;
+                        o.x = prmt(p0, p1, 0x5410);   // k 0, 1
+                        o.y = prmt(p2, p3, 0x5410);   // k 2, 3
+                        o.z = prmt(p0, p1, 0x7632);   // k 4, 5
+                        o.w = prmt(p2, p3, 0x7632);   // k 6, 7
+                        *reinterpret_cast<uint4 *>(arow + ((j ^ (i & 7)) << 4)) = o;
+                    }
+                    fence_proxy_async_smem();
+                }
+                mbar_arrive(aready0 + 8 * slot);
+            }
+            if (!ok)
+                break;
+        }
+    } else {
+        // ------------------------------------------------ epilogue: warp quarter q owns TMEM lanes 32q..32q+31
+        const int q = warp & 3;
+        const int row = 32 * q + lane;
+        int lt = 0;
+        for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++lt) {
+            const uint32_t buf = lt & 1;
+            if (!mbar_wait(tfull0 + 8 * buf, (lt >> 1) & 1, &abort_flag, p.status))
+                break;
+            tc_fence_after();
+            const int64_t t0 = (int64_t)(tile % p.n_ttiles) * BN;
+            const int64_t n = (int64_t)(tile / p.n_ttiles) * BM + row;
+            const float sn = p.s[n];
+            const float e_n = sn != 0.0f ? sn : 1.0f;   // the EC operand was divided by it
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * BN + 32 * c, r);
+                if (n < p.N) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int64_t t = t0 + 32 * c + j;
+                        if (t < p.M)
+                            p.y[t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(e_n * __uint_as_float(r[j])));
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(tempty0 + 8 * buf);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace
+
+bool tc_available(const Packed &) { return tensor_maps_available(); }
+
+cudaError_t tc_alloc(const Packed &, int64_t, int, TcWork &w)
+{
+    w.maps = new (std::nothrow) Maps();
+    return w.maps ? cudaSuccess : cudaErrorMemoryAllocation;
+}
+
+void tc_free(TcWork &w)
+{
+    delete static_cast<Maps *>(w.maps);
+    w.maps = nullptr;
+}
+
+cudaError_t tc_prepare(const Packed &pk, TcWork &w)
+{
+    Maps *m = static_cast<Maps *>(w.maps);
+    if (!m)
+        return cudaErrorInvalidValue;
+    cudaError_t e = make_map(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)pk.Kp / 8,
+                             (uint64_t)pk.Np, BK / 8, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e == cudaSuccess && pk.r > 0)
+        e = make_map(&m->bt, pk.Bts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.rp, (uint64_t)pk.Np, BK, BM,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+    return e;
+}
+
+cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const uint16_t *v, bool ec,
+                      const TcWork &w, int *status, bool zero_wait_budget, cudaStream_t st, int num_sms)
+{
+    if (M <= 0)
+        return cudaSuccess;
+    const Maps *m = static_cast<const Maps *>(w.maps);
+    if (!m)
+        return cudaErrorInvalidValue;
+    if (zero_wait_budget) {
+        // injected fault: report what a wait that ran out reports, launch nothing
+        const int bits = kStatusTimeout;
+        return cudaMemcpyAsync(status, &bits, sizeof(int), cudaMemcpyHostToDevice, st);
+    }
+    CUtensorMap tm_x, tm_v;
+    cudaError_t e = make_map(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.K, (uint64_t)M, BK, BN,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess)
+        return e;
+    const bool use_ec = ec && pk.r > 0;
+    if (use_ec) {
+        e = make_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.rp, (uint64_t)M, BK, BN,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+        if (e != cudaSuccess)
+            return e;
+    } else {
+        tm_v = tm_x;  // unused
+    }
+    TcParams p;
+    p.M = M;
+    p.N = pk.N;
+    p.n_main = (int)(pk.Kp / BK);
+    p.n_ec = use_ec ? (pk.rp + BK - 1) / BK : 0;
+    p.rp = pk.rp;
+    p.n_ttiles = (int)((M + BN - 1) / BN);
+    p.n_tiles = p.n_ttiles * (int)(pk.Np / BM);
+    p.s = pk.s;
+    p.z = pk.z;
+    p.y = static_cast<uint16_t *>(y);
+    p.status = status;
+
+    e = raise_smem_limit(reinterpret_cast<const void *>(tc_w4ec_kernel), SMEM_BYTES);
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.n_tiles < num_sms ? p.n_tiles : num_sms));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc_w4ec_kernel, tm_x, m->codes, use_ec ? m->bt : m->codes, tm_v, p);
 }
 
 }  // namespace spear
