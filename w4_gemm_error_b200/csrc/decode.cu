@@ -46,7 +46,7 @@ constexpr int kMaxChunks = 8;   // so K/CS <= 2048
 constexpr int kUStride = 32;    // token stride of the published u rows
 
 struct Maps {
-    CUtensorMap codes;  // [Np][Kp/8] u32, boxes of 32 words x 64 rows, 128B swizzle
+    CUtensorMap codes;  // tiled codes, one box = one 8 KB block (64 rows x 256 k), 128B swizzle
     CUtensorMap g;      // [R1p][Kp] bf16, boxes of 64 x 16, 128B swizzle
     CUtensorMap bt;     // [Np][rp] bf16, boxes of rp x 64
 };
@@ -145,7 +145,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                     tma_load_2d(base + L.codes + c * 8192 + i * 2048, &tm_g, k0 + c * kChunk + i * 64, 16 * cluster,
                                 bar);
             } else {
-                tma_load_2d(base + L.codes + c * 8192, &tm_codes, (k0 + c * kChunk) / 8, n0, bar);
+                tma_load_3d(base + L.codes + c * 8192, &tm_codes, 0, 0,
+                            (n0 / kRows) * (int)(p.Kp / kChunk) + (k0 / kChunk) + c, bar);
             }
         }
         // the activations are written by the previous kernel in the stream
@@ -429,8 +430,12 @@ cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
             return cudaErrorMemoryAllocation;
         w.maps = m;
     }
-    cudaError_t e = make_map(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)pk.Kp / 8,
-                             (uint64_t)pk.Np, 32, kRows, CU_TENSOR_MAP_SWIZZLE_128B);
+    // [blocks][64 rows][32 words]: one box = one contiguous 8 KB block of 64 rows x 256 k
+    const uint64_t dims[3] = {32, (uint64_t)kRows, (uint64_t)(pk.Np / kRows) * (uint64_t)(pk.Kp / kChunk)};
+    const uint64_t strides[2] = {128, 8192};
+    const uint32_t box[3] = {32, (uint32_t)kRows, 1};
+    cudaError_t e = make_map_nd(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, dims, strides, box,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
     if (e == cudaSuccess && pk.r > 0)
         e = make_map(&m->g, pk.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.Kp, (uint64_t)pk.R1p, 64, 16,
                      CU_TENSOR_MAP_SWIZZLE_128B);

@@ -10,7 +10,10 @@ namespace spear {
 cudaError_t raise_smem_limit(const void *func, size_t bytes);
 
 // Library-owned packed layout (all device memory, zero/neutral padded):
-//   codes [Np][Kp/8] uint32   code of k = 8j+i in bits [4i,4i+3] of word j;
+//   codes tiled [Np/64][Kp/256][64][32] uint32: the word holding codes k = 8j..8j+7
+//                             of row n (code of k = 8j+i in bits [4i,4i+3]) sits at
+//                             ((n/64 * Kp/256 + j/32) * 64 + n%64) * 32 + j%32, so every
+//                             64-row x 256-k block is 8 KB of contiguous memory;
 //                             padding words hold code 8 (weight 0)
 //   s     [Np] float          per-channel scale (0 on padding rows)
 //   z     [Np] uint8          per-channel zero point (8)
@@ -36,6 +39,8 @@ struct Packed {
 // ---- pack: per-channel RTN int4 of W, plus the EC operand layouts
 cudaError_t launch_pack(const Packed &pk, const void *W, const void *A, const void *B,
                         const void *wg, int *status, cudaStream_t st);
+// codes in the exported layout [N][K/8] (row-major, no padding)
+cudaError_t launch_untile_codes(const Packed &pk, uint32_t *dst, cudaStream_t st);
 
 // Every forward-pass kernel is launched with programmatic dependent launch:
 // it lets its own dependents start at once and waits for its predecessor

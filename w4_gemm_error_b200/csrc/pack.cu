@@ -8,7 +8,9 @@
 //   s[n] = fp32(max_k |W[n,k]|) / 7        (IEEE fp32 division)
 //   q    = clamp(rint(fp32(W[n,k] / s[n])), -8, 7) + 8    (ties to even)
 //   z[n] = 8;  an all-zero row has s = 0 and every code 8
-//   code of k = 8j+i in bits [4i, 4i+3] of word j of row n.
+//   code of k = 8j+i in bits [4i, 4i+3] of word j of row n (exported
+//   layout [N][K/8]; stored tiled in 8 KB blocks of 64 rows x 256 k, see
+//   kernels.h).
 #include "device_utils.cuh"
 #include "kernels.h"
 
@@ -27,10 +29,12 @@ pack_w4_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K, int64_t Np,
     if (row >= Np)
         return;
     const int64_t words = Kp / 8, valid_words = K / 8;
-    uint32_t *crow = codes + row * words;
+    // tiled layout: word j of row n at ((n/64 * Kp/256 + j/32) * 64 + n%64) * 32 + j%32
+    uint32_t *crow = codes + ((row >> 6) * (Kp / 256) * 64 + (row & 63)) * 32;
+    auto word_at = [&](int64_t j) -> uint32_t & { return crow[(j >> 5) * 64 * 32 + (j & 31)]; };
     if (row >= N) {
         for (int64_t j = lane; j < words; j += 32)
-            crow[j] = 0x88888888u;
+            word_at(j) = 0x88888888u;
         if (lane == 0) {
             s[row] = 0.0f;
             z[row] = 8;
@@ -73,7 +77,7 @@ pack_w4_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K, int64_t Np,
                 word |= (uint32_t)((int)c + 8) << (4 * i);
             }
         }
-        crow[j] = word;
+        word_at(j) = word;
     }
     if (lane == 0) {
         s[row] = sn;
@@ -116,7 +120,24 @@ __global__ void pack_ec_kernel(const uint16_t *__restrict__ A, const uint16_t *_
     }
 }
 
+__global__ void untile_codes_kernel(const uint32_t *__restrict__ tiled, uint32_t *__restrict__ dst, int64_t N,
+                                    int64_t K, int64_t Kp)
+{
+    const int64_t words = K / 8;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < N * words;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = i / words, j = i - n * words;
+        dst[i] = tiled[(((n >> 6) * (Kp / 256) + (j >> 5)) * 64 + (n & 63)) * 32 + (j & 31)];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_untile_codes(const Packed &pk, uint32_t *dst, cudaStream_t st)
+{
+    untile_codes_kernel<<<1024, 256, 0, st>>>(pk.codes, dst, pk.N, pk.K, pk.Kp);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_pack(const Packed &pk, const void *W, const void *A, const void *B,
                         const void *wg, int *status, cudaStream_t st)

@@ -390,8 +390,7 @@ int spear_w4ec_get_packed(const spear_w4ec *h, void *codes, float *s, uint8_t *z
     const Packed &pk = h->pk;
     cudaError_t e = cudaSuccess;
     if (codes)
-        e = cudaMemcpy2DAsync(codes, (size_t)pk.K / 2, pk.codes, (size_t)pk.Kp / 2, (size_t)pk.K / 2, (size_t)pk.N,
-                              cudaMemcpyDeviceToDevice, st);
+        e = launch_untile_codes(pk, static_cast<uint32_t *>(codes), st);
     if (e == cudaSuccess && s)
         e = cudaMemcpyAsync(s, pk.s, (size_t)pk.N * sizeof(float), cudaMemcpyDeviceToDevice, st);
     if (e == cudaSuccess && z)

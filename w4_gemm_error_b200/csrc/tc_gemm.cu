@@ -56,6 +56,7 @@ constexpr int TMEM_COLS = 2 * BN;
 
 struct TcParams {
     int64_t M, N;
+    int kchunks;       // Kp / 256: tiled code blocks per 64-row block
     int n_main, n_ec, rp;
     int n_ttiles, n_tiles;
     const float *s;
@@ -137,7 +138,10 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     if (st < p.n_main) {
                         mbar_expect_tx(full, B_BYTES + C_BYTES);
                         tma_load_2d(sb + A_BYTES, &tm_x, st * BK, t0, full);
-                        tma_load_2d(sb + A_BYTES + B_BYTES, &tm_codes, st * (BK / 8), n0, full);
+                        const int blk = (n0 / 64) * p.kchunks + st / 4;
+                        tma_load_4d(sb + A_BYTES + B_BYTES, &tm_codes, 0, st & 3, 0, blk, full);
+                        tma_load_4d(sb + A_BYTES + B_BYTES + C_BYTES / 2, &tm_codes, 0, st & 3, 0, blk + p.kchunks,
+                                    full);
                     } else {
                         const int e = st - p.n_main;
                         mbar_expect_tx(full, A_BYTES + B_BYTES);
@@ -296,8 +300,13 @@ cudaError_t tc_prepare(const Packed &pk, TcWork &w)
     Maps *m = static_cast<Maps *>(w.maps);
     if (!m)
         return cudaErrorInvalidValue;
-    cudaError_t e = make_map(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)pk.Kp / 8,
-                             (uint64_t)pk.Np, BK / 8, BM, CU_TENSOR_MAP_SWIZZLE_NONE);
+    // tiled codes viewed as [blocks][64 rows][4 sub-chunks][8 words]: a box is the 32 bytes
+    // (64 k) of one sub-chunk of 64 rows; two boxes (row blocks) make the 128-row stage
+    const uint64_t dims[4] = {8, 4, 64, (uint64_t)(pk.Np / 64) * (uint64_t)(pk.Kp / 256)};
+    const uint64_t strides[3] = {32, 128, 8192};
+    const uint32_t box[4] = {8, 1, 64, 1};
+    cudaError_t e = make_map_nd(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, dims, strides, box,
+                                CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e == cudaSuccess && pk.r > 0)
         e = make_map(&m->bt, pk.Bts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.rp, (uint64_t)pk.Np, BK, BM,
                      CU_TENSOR_MAP_SWIZZLE_128B);
@@ -334,6 +343,7 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
     TcParams p;
     p.M = M;
     p.N = pk.N;
+    p.kchunks = (int)(pk.Kp / 256);
     p.n_main = (int)(pk.Kp / BK);
     p.n_ec = use_ec ? (pk.rp + BK - 1) / BK : 0;
     p.rp = pk.rp;
