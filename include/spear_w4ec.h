@@ -137,6 +137,28 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
 /* The flags (path | fused/split) that forward would use for M tokens now. */
 int spear_w4ec_dispatch(const spear_w4ec *h, int64_t M, uint32_t *choice);
 
+/* Per-token gate with no allocation at all, for callers that may not call
+ * cudaMalloc (code inside a CUDA graph capture, a real-time serving loop with
+ * a fixed memory budget, a host framework whose pool owns every allocation):
+ *   g[t] = 1 / (1 + exp(-(x[t,:] . w_g + b_g)))   for t < M,
+ * the same gate as spear_w4ec_get_gate, from the caller's own buffers and
+ * without a handle.  (The SPEAR pages have no counterpart of this call; it
+ * exists for those callers.)
+ *   x    dev bf16 [M][K], 16-byte aligned;  w_g  dev bf16 [K], 16-byte aligned
+ *   g    dev float [M]
+ * K must be a positive multiple of 8 and 0 <= M <= 4096; a larger M returns
+ * SPEAR_ERR_INVALID (the scratch is sized for 4096 tokens).  Runs on the
+ * current device and `stream`.
+ * Scratch: one static device array of 65,536 + 1,024 bytes inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits.  All calls share it and each call clears the part that must start
+ * at zero, so calls that overlap on the GPU (different streams without
+ * ordering between them) race and must be avoided.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress); make
+ * that first call before any stream capture. */
+int spear_w4ec_gate_noalloc(const void *x, int64_t M, int64_t K, const void *w_g, float b_g, float *g,
+                            void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *spear_w4ec_strerror(int status);
 

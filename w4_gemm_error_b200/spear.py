@@ -32,7 +32,7 @@ SPEAR_FORCE_TC = 16
 
 EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_forward", "spear_w4ec_forward_host",
             "spear_w4ec_destroy", "spear_w4ec_get_packed", "spear_w4ec_get_gate", "spear_w4ec_sync_status",
-            "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_strerror")
+            "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_gate_noalloc", "spear_w4ec_strerror")
 
 
 class SpearError(RuntimeError):
@@ -61,6 +61,7 @@ def _load():
         "spear_w4ec_sync_status": [P, P],
         "spear_w4ec_tune": [P, P, P, i64, P, ctypes.POINTER(u32)],
         "spear_w4ec_dispatch": [P, i64, ctypes.POINTER(u32)],
+        "spear_w4ec_gate_noalloc": [P, i64, i64, P, f32, P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -153,6 +154,12 @@ def spear_w4ec_dispatch(h: int, M: int) -> int:
     choice = ctypes.c_uint32(0)
     _check(_lib.spear_w4ec_dispatch(h, M, ctypes.byref(choice)), "spear_w4ec_dispatch")
     return choice.value
+
+
+def spear_w4ec_gate_noalloc(x, M: int, K: int, w_g, b_g: float, g, stream=None):
+    """Gate g[t] for M <= 4096 tokens with no allocation (static scratch inside the library)."""
+    _check(_lib.spear_w4ec_gate_noalloc(_ptr(x), M, K, _ptr(w_g), float(b_g), _ptr(g), _stream(stream)),
+           "spear_w4ec_gate_noalloc")
 
 
 class W4ECLinear:
