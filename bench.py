@@ -48,6 +48,20 @@ WORKLOADS = {
 }
 
 
+def reduce_over_ranks(ms: float, units: float, world: int, device=None):
+    """Whole-job figures of a replicas run: the slowest rank's time and the
+    units all ranks processed (every rank does the same work)."""
+    if world <= 1:
+        return ms, units
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
 def alg_bytes(M, K, N, r):
     """Bytes the method must move for one forward (no split-K partials, no padding)."""
     return N * K // 2 + 4 * N + N + 2 * K * r + 2 * r * N + 2 * K + 2 * M * K + 2 * M * N
@@ -207,11 +221,8 @@ def run_ours(args, rank, world, local_rank):
                 e1.record(stream)
             e1.synchronize()
         torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1)
+        ms, _ = reduce_over_ranks(e0.elapsed_time(e1), 0.0, world, dev)
         if world > 1:
-            t = torch.tensor([ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
             dist.barrier()
         return ms, (sampler.summary() if sampler else None)
 
@@ -228,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
     else:
         units_per_step = sum(alg_flops(M, K, N, r) for M in Ms) * L
         unit, scale = "TFLOP/s", 1e12
-    total_units = units_per_step * args.steps * world
+    _, total_units = reduce_over_ranks(0.0, float(units_per_step * args.steps), world, dev)
     value = total_units / (ms_on * 1e-3) / scale
     per_gpu = value / world
     ms_per_step = ms_on / args.steps
@@ -260,13 +271,8 @@ def run_ours(args, rank, world, local_rank):
     t0 = time.perf_counter()
     for _ in range(e2e_steps):
         e2e_step()
-    e2e_s = time.perf_counter() - t0
-    if world > 1:
-        import torch as _t
-        tt = _t.tensor([e2e_s], device=dev, dtype=_t.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_s = float(tt.item())
-    e2e_value = units_per_step * e2e_steps * world / e2e_s / scale
+    e2e_s, e2e_units = reduce_over_ranks(time.perf_counter() - t0, float(units_per_step * e2e_steps), world, dev)
+    e2e_value = e2e_units / e2e_s / scale
     h2d = sum(M * K * 2 for M in Ms)
     d2h = sum(M * N * 2 for M in Ms)
 

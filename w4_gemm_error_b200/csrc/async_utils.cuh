@@ -10,8 +10,10 @@
 
 namespace spear {
 
-// Bounded waits give up after about this long (a second of %globaltimer).
-constexpr unsigned long long kWaitBudgetNs = 1000000000ull;
+// Bounded waits give up after about this long: 2^31 SM clock cycles, about a
+// second at the B200's 1.9 GHz (the SM cycle counter is cheap to read, unlike
+// %globaltimer).
+constexpr long long kWaitBudgetCycles = 1LL << 31;
 
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
@@ -59,13 +61,13 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 {
     if (mbar_try_wait(bar, parity))
         return true;
-    const unsigned long long t0 = globaltimer();
+    const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity))
             return true;
         if (*abort_flag)
             return false;
-        if (globaltimer() - t0 > kWaitBudgetNs) {
+        if (clock64() - t0 > kWaitBudgetCycles) {
             *abort_flag = 1;
             atomicOr(status, kStatusTimeout);
             return false;
@@ -73,13 +75,23 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Bounded wait without a shared abort flag: false if it runs out.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity))
+        if (clock64() - t0 > kWaitBudgetCycles)
+            return false;
+    return true;
+}
+
 // Teardown wait: bounded, and kept even after the CTA has given up, so that
 // no copy or MMA is still writing when the CTA releases its memory.
 __device__ __forceinline__ void mbar_wait_final(uint32_t bar, uint32_t parity)
 {
-    const unsigned long long t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity) && globaltimer() - t0 < kWaitBudgetNs) {
-    }
+    mbar_wait_bounded(bar, parity);
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1, uint32_t bar)
@@ -135,6 +147,17 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }

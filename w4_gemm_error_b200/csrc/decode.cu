@@ -11,9 +11,11 @@
 //    CTA one K/CS slice of them;
 //  * before waiting for the previous kernel (programmatic dependent launch)
 //    every CTA starts TMA copies of its whole slice of codes (and the
-//    cluster's first CTA loads the scales and B^T rows of its epilogue into
-//    registers), so the weight stream overlaps the previous layer; only the
-//    activations are fetched after the wait;
+//    cluster's first CTA those of the B^T rows of its epilogue), so the
+//    weight stream overlaps the previous layer; only the activations are
+//    fetched after the wait;
+//  * eight warps per CTA, two per 16-row group splitting the 64-wide
+//    sub-blocks, so the dequantise-MMA chains of one warp hide another's;
 //  * weight rows sit on the 16-row side of mma.sync m16n8k16 and tokens on
 //    the 8-column side, so a code is read once for up to 32 tokens; the
 //    codes are dequantised in registers to exact (q - z) bf16 pairs (two
@@ -46,9 +48,9 @@ constexpr int kMaxChunks = 8;   // so K/CS <= 2048
 constexpr int kUStride = 32;    // token stride of the published u rows
 
 struct Maps {
-    CUtensorMap codes;  // tiled codes, one box = one 8 KB block (64 rows x 256 k), 128B swizzle
-    CUtensorMap g;      // [R1p][Kp] bf16, boxes of 64 x 16, 128B swizzle
-    CUtensorMap bt;     // [Np][rp] bf16, boxes of rp x 64
+    CUtensorMap codes;    // tiled codes, one box = one 8 KB block (64 rows x 256 k), 128B swizzle
+    CUtensorMap g;        // [R1p][Kp] bf16, boxes of 64 x 16, 128B swizzle
+    CUtensorMap bt;       // [Np][rp] bf16, boxes of rp x 64
 };
 
 struct DecodeParams {
@@ -78,23 +80,18 @@ __host__ __device__ inline Smem smem_layout(int KS, int rp, int R1p)
     m.codes = 0;                                   // 32*KS bytes: codes (64 rows) or G (16 rows bf16)
     m.x = m.codes + 32 * KS;                       // 2*TOK*KS bytes: activation sub-tiles
     m.bt = m.x + 2 * TOK * KS;                     // 128*rp bytes: B^T rows of the cluster
-    m.red = m.bt + 128 * rp;                       // 256*TOK bytes: partial tile
-    m.u = m.red + 256 * TOK;                       // u [R1p][TOK], g [TOK], v [TOK][rp] (fp32)
+    m.red = m.bt + 128 * rp;                       // 512*TOK bytes: partial tiles
+    m.u = m.red + 512 * TOK;                       // u [R1p][TOK], g [TOK], v [TOK][rp] (fp32)
     m.total = m.u + 4 * R1p * TOK + 4 * TOK * (rp + 1);
     return m;
 }
 
-__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity)
-{
-    const unsigned long long t0 = globaltimer();
-    while (!mbar_try_wait(bar, parity))
-        if (globaltimer() - t0 > kWaitBudgetNs)
-            return false;
-    return true;
-}
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) { return mbar_wait_bounded(bar, parity); }
+
+constexpr int kThreads = 256;   // 8 warps: two per 16-row group, splitting the sub-blocks
 
 template <int T>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kThreads)
 decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_g,
                    const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_x,
                    DecodeParams p, int CS)
@@ -122,16 +119,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     const uint32_t bar_bt = smem_addr(&bars[kMaxChunks + 1]);
     const int n0 = is_u ? 0 : (cluster - p.JB) * kRows;
 
-    // epilogue operands of this thread's row, requested before anything else
-    float s_epi = 0.f;
-    uint4 bt_pre[8];
-    if (!is_u && rank == 0) {
-        const int64_t n_epi = n0 + (tid & (kRows - 1));
-        s_epi = __ldg(p.s + n_epi);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            bt_pre[q] = (8 * q < p.rp) ? ld_nc(p.Bt + n_epi * p.rp + 8 * q) : make_uint4(0, 0, 0, 0);
-    }
+    // epilogue scale of this thread's row, requested before anything else
+    const float s_epi = (!is_u && rank == 0) ? __ldg(p.s + n0 + (tid & (kRows - 1))) : 0.f;
     if (tid == 0) {
         for (int c = 0; c < kMaxChunks + 2; ++c)
             mbar_init(bar_chunk + 8 * c, 1);
@@ -148,6 +137,10 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 tma_load_3d(base + L.codes + c * 8192, &tm_codes, 0, 0,
                             (n0 / kRows) * (int)(p.Kp / kChunk) + (k0 / kChunk) + c, bar);
             }
+        }
+        if (!is_u && rank == 0 && p.rp > 0) {
+            mbar_expect_tx(bar_bt, 128 * p.rp);   // B^T rows of the cluster, for the epilogue
+            tma_load_2d(base + L.bt, &tm_bt, 0, n0, bar_bt);
         }
         // the activations are written by the previous kernel in the stream
         pdl_wait();
@@ -168,8 +161,9 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 
     float *red = reinterpret_cast<float *>(bp + L.red);
     if (!is_u) {
-        // ---- 64 weight rows: warp w owns rows 16w .. 16w+15
-        const int rg = 16 * warp + gid;  // and rg + 8 (same row mod 8)
+        // ---- 64 weight rows: warps w and w+4 own rows 16w .. 16w+15, sub-blocks of parity w>>2
+        const int rg = 16 * (warp & 3) + gid;  // and rg + 8 (same row mod 8)
+        const int kpar = warp >> 2;
         const uint32_t zg = 128u + p.z[n0 + rg], zh = 128u + p.z[n0 + rg + 8];
         const uint32_t nbg = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)zg));
         const uint32_t nbh = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)zh));
@@ -178,7 +172,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             ok = wait_bounded(bar_chunk + 8 * c, 0);
             const uint8_t *ctile = bp + L.codes + c * 8192;
 #pragma unroll
-            for (int sb = 0; sb < 4; ++sb) {
+            for (int sb2 = 0; sb2 < 2; ++sb2) {
+                const int sb = 2 * sb2 + kpar;
                 // codes k = 64 sb + 16 cl + {0..15} of rows rg and rg + 8 (8 bytes each)
                 const int chunk = ((2 * sb + (cl >> 1)) ^ (rg & 7)) * 16 + (cl & 1) * 8;
                 const uint2 wgv = *reinterpret_cast<const uint2 *>(ctile + rg * 128 + chunk);
@@ -208,17 +203,21 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 }
             }
         }
+        float *mine = red + kpar * kRows * TOK;   // [2][64][TOK]
 #pragma unroll
         for (int n = 0; n < T; ++n) {
             const int col = 8 * n + 2 * cl;
-            red[rg * TOK + col] = acc[n][0];
-            red[rg * TOK + col + 1] = acc[n][1];
-            red[(rg + 8) * TOK + col] = acc[n][2];
-            red[(rg + 8) * TOK + col + 1] = acc[n][3];
+            mine[rg * TOK + col] = acc[n][0];
+            mine[rg * TOK + col + 1] = acc[n][1];
+            mine[(rg + 8) * TOK + col] = acc[n][2];
+            mine[(rg + 8) * TOK + col + 1] = acc[n][3];
         }
+        __syncthreads();
+        for (int e = tid; e < kRows * TOK; e += kThreads)
+            red[e] = red[e] + red[kRows * TOK + e];
     } else {
-        // ---- 16 rows of G = [w_g; A^T]: warp w takes the 64-wide sub-tiles i = w (mod 4)
-        for (int i = warp; i < nsub && ok; i += 4) {
+        // ---- 16 rows of G = [w_g; A^T]: warp w takes the 64-wide sub-tiles i = w (mod 8)
+        for (int i = warp; i < nsub && ok; i += 8) {
             ok = wait_bounded(bar_chunk + 8 * (i >> 2), 0);
             const uint8_t *gt = bp + L.codes + i * 2048;
             const uint8_t *xt = bp + L.x + i * (TOK * 128);
@@ -242,7 +241,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                                    xa[2 * s + 1]);
             }
         }
-        float *mine = red + warp * 16 * TOK;  // [4 warps][16][TOK]
+        float *mine = red + warp * 16 * TOK;  // [8 warps][16][TOK]
 #pragma unroll
         for (int n = 0; n < T; ++n) {
             const int col = 8 * n + 2 * cl;
@@ -252,8 +251,13 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             mine[(gid + 8) * TOK + col + 1] = acc[n][3];
         }
         __syncthreads();
-        for (int e = tid; e < 16 * TOK; e += 128)
-            red[e] = red[e] + red[16 * TOK + e] + red[32 * TOK + e] + red[48 * TOK + e];
+        for (int e = tid; e < 16 * TOK; e += kThreads) {
+            float s = red[e];
+#pragma unroll
+            for (int w = 1; w < 8; ++w)
+                s += red[w * 16 * TOK + e];
+            red[e] = s;
+        }
     }
     if (!ok)
         atomicOr(p.status, kStatusTimeout);
@@ -264,6 +268,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         for (int c = 0; c < nch; ++c)
             wait_bounded(bar_chunk + 8 * c, 0);
         wait_bounded(bar_x, 0);
+        if (!is_u && rank == 0 && p.rp > 0)
+            wait_bounded(bar_bt, 0);
     }
 
     // ---- sum the K split over the cluster, in rank order, in the first CTA
@@ -272,7 +278,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     const int tile = (is_u ? 16 : kRows) * TOK;
     if (rank == 0) {
         const uint32_t red_addr = base + L.red;
-        for (int e4 = tid; e4 < tile / 4; e4 += 128) {
+        for (int e4 = tid; e4 < tile / 4; e4 += kThreads) {
             // issue every remote load before summing (in rank order)
             float4 o[8];
 #pragma unroll
@@ -298,7 +304,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 
     if (is_u) {
         // publish u rows 16*cluster .. +15 for all TOK token columns
-        for (int e = tid; e < 16 * TOK; e += 128) {
+        for (int e = tid; e < 16 * TOK; e += kThreads) {
             const int row = e / TOK, t = e - row * TOK;
             p.ws_u[(16 * cluster + row) * kUStride + t] = red[e];
         }
@@ -316,9 +322,9 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     if (p.JB > 0) {
         if (tid == 0) {
             int good = 1;
-            const unsigned long long t0 = globaltimer();
+            const long long t0 = clock64();
             while (ld_acquire_gpu(&p.flags[0]) < (unsigned)p.JB) {
-                if (globaltimer() - t0 > kWaitBudgetNs) {
+                if (clock64() - t0 > kWaitBudgetCycles) {
                     atomicOr(p.status, kStatusTimeout);
                     good = 0;
                     break;
@@ -328,7 +334,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             s_ok = good;
         }
         __syncthreads();
-        for (int e = tid; e < p.R1p * TOK; e += 128) {
+        for (int e = tid; e < p.R1p * TOK; e += kThreads) {
             const int row = e / TOK, t = e - row * TOK;
             us[e] = s_ok ? __ldcg(p.ws_u + row * kUStride + t) : 0.f;
         }
@@ -341,52 +347,46 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         if (tid < TOK)
             gs[tid] = 1.0f / (1.0f + expf(-(us[tid] + p.b_g)));
         __syncthreads();
-        for (int e = tid; e < TOK * p.rp; e += 128) {
+        for (int e = tid; e < TOK * p.rp; e += kThreads) {
             const int t = e / p.rp, j = e - t * p.rp;
             vv[e] = j < p.r ? gs[t] * us[(1 + j) * TOK + t] : 0.f;
         }
+        if (!wait_bounded(bar_bt, 0))
+            atomicOr(p.status, kStatusTimeout);
         __syncthreads();
     }
 
-    const int row = tid & (kRows - 1), th = tid >> 6;
+    const int row = tid & (kRows - 1), th = tid >> 6;  // four token phases
     const int64_t n = n0 + row;
-    float out[TOK / 2];
+    float out[TOK / 4];
 #pragma unroll
-    for (int i = 0; i < TOK / 2; ++i)
-        out[i] = s_epi * red[row * TOK + th + 2 * i];
+    for (int i = 0; i < TOK / 4; ++i)
+        out[i] = s_epi * red[row * TOK + th + 4 * i];
     if (p.JB > 0) {
-        // corr = sum_j v[t][j] * B^T[n][j]: B^T row in registers (8 values per 16 bytes),
+        // corr = sum_j v[t][j] * B^T[n][j]: the B^T row in 16-byte pieces from shared memory,
         // v broadcast from shared memory
-        const uint16_t *btg = p.Bt + n * p.rp;
-        auto accumulate = [&](int j0, const uint4 bv) {
+        const uint16_t *btrow = reinterpret_cast<const uint16_t *>(bp + L.bt) + row * p.rp;
+        for (int j0 = 0; j0 < p.rp; j0 += 8) {
+            const uint4 bv = *reinterpret_cast<const uint4 *>(btrow + j0);
             const float bj[8] = {bf16_lo(bv.x), bf16_hi(bv.x), bf16_lo(bv.y), bf16_hi(bv.y),
                                  bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
 #pragma unroll
-            for (int i = 0; i < TOK / 2; ++i) {
-                const float4 *vt = reinterpret_cast<const float4 *>(vv + (th + 2 * i) * p.rp + j0);
+            for (int i = 0; i < TOK / 4; ++i) {
+                const float4 *vt = reinterpret_cast<const float4 *>(vv + (th + 4 * i) * p.rp + j0);
                 const float4 v0 = vt[0], v1 = vt[1];
                 out[i] += v0.x * bj[0] + v0.y * bj[1] + v0.z * bj[2] + v0.w * bj[3] + v1.x * bj[4] +
                           v1.y * bj[5] + v1.z * bj[6] + v1.w * bj[7];
             }
-        };
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            if (8 * q < p.rp)
-                accumulate(8 * q, bt_pre[q]);
-        for (int j0 = 64; j0 < p.rp; j0 += 8)
-            accumulate(j0, ld_nc(btg + j0));
+        }
     }
 #pragma unroll
-    for (int i = 0; i < TOK / 2; ++i) {
-        const int t = th + 2 * i;
+    for (int i = 0; i < TOK / 4; ++i) {
+        const int t = th + 4 * i;
         if (t < p.M && n < p.N)
             p.y[(int64_t)t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
     }
 }
 
-// Cluster size CS (CTAs splitting K) and the k per CTA, or 0 if a slice would
-// not fit in shared memory.  Up to 8 CTAs per cluster, fewer when the grid
-// would exceed about 8 CTAs per SM.
 int pick_cluster(const Packed &pk, int num_sms, int JB, int *KS_out)
 {
     const int NC = (int)(pk.Np / kRows);
@@ -436,12 +436,14 @@ cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
     const uint32_t box[3] = {32, (uint32_t)kRows, 1};
     cudaError_t e = make_map_nd(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, dims, strides, box,
                                 CU_TENSOR_MAP_SWIZZLE_128B);
+
     if (e == cudaSuccess && pk.r > 0)
         e = make_map(&m->g, pk.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.Kp, (uint64_t)pk.R1p, 64, 16,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     if (e == cudaSuccess && pk.r > 0)
         e = make_map(&m->bt, pk.Bt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.rp, (uint64_t)pk.Np,
                      (uint32_t)pk.rp, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+
     if (e == cudaSuccess && pk.r == 0) {
         m->g = m->codes;
         m->bt = m->codes;
@@ -505,7 +507,7 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((p.JB + p.NC) * CS));
-    cfg.blockDim = dim3(128);
+    cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];

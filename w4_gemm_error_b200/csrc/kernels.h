@@ -19,9 +19,9 @@ cudaError_t raise_smem_limit(const void *func, size_t bytes);
 //   z     [Np] uint8          per-channel zero point (8)
 //   G     [R1p][Kp] bf16      row 0 = w_g, rows 1..r = A^T, other rows 0
 //   Bt    [Np][rp] bf16       B transposed (Bt[n][j] = B[j][n]), zero padded
-//   Bts   [Np][rp] bf16       Bt[n][j] / e[n] with e[n] = s[n] (1 where s[n] = 0): the EC
-//                             operand of kernels that accumulate sum_k x (q - z) unscaled
-//                             and apply e[n] once at the end
+//   Bts   [Np][rp] fp32       Bt[n][j] / e[n] rounded to tf32, e[n] = s[n] (1 where
+//                             s[n] = 0): the EC operand of the tcgen05 kernel, which
+//                             accumulates sum_k x (q - z) unscaled and applies e[n] once
 // Np = N rounded up to 128, Kp = K rounded up to 256, rp = r rounded up to 16,
 // R1p = (r + 1) rounded up to 16.
 struct Packed {
@@ -32,7 +32,7 @@ struct Packed {
     uint8_t *z;
     uint16_t *G;
     uint16_t *Bt;
-    uint16_t *Bts;
+    float *Bts;
     float b_g;
 };
 
@@ -47,15 +47,15 @@ cudaError_t launch_untile_codes(const Packed &pk, uint32_t *dst, cudaStream_t st
 // (griddepcontrol.wait) before reading anything a previous kernel wrote.
 
 // ---- prepass: per-token gate and EC down-projection
-//   g[t] = sigmoid(x[t].w_g + b_g),  v[t][j] = bf16(g[t] * x[t].A[:,j])  (v is [M][rp])
+//   g[t] = sigmoid(x[t].w_g + b_g),  v[t][j] = g[t] * x[t].A[:,j]  (v is fp32 [M][rp],
+//   rounded to tf32 when `tf32` is set: the operand of the tcgen05 kernel's EC k-steps)
 struct PrepassWork {
     float *part;          // split-K partials
     size_t part_floats;
     unsigned *counters;   // one per 16-token tile, zero between calls
     int n_counters;
 };
-// vf (may be null) receives v in fp32 [M][rp] for kernels that do not need a bf16 operand.
-cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t *v, float *vf, float *g,
+cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
                            const PrepassWork &w, cudaStream_t st, int num_sms);
 size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms);
 int prepass_counters(int64_t max_M);

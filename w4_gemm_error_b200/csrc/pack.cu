@@ -86,11 +86,11 @@ pack_w4_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K, int64_t Np,
 }
 
 // G [R1p][Kp]: row 0 = w_g, rows 1..r = A^T;  Bt [Np][rp] = B^T; zeros elsewhere.
-// Bts = Bt / e[n], e[n] = s[n] (1 where s[n] = 0), in fp32 rounded once to bf16.
+// Bts = Bt / e[n], e[n] = s[n] (1 where s[n] = 0): fp32 quotient rounded to tf32.
 __global__ void pack_ec_kernel(const uint16_t *__restrict__ A, const uint16_t *__restrict__ B,
                                const uint16_t *__restrict__ wg, const float *__restrict__ s, int64_t K,
                                int64_t N, int r, int64_t Kp, int64_t Np, int R1p, int rp,
-                               uint16_t *__restrict__ G, uint16_t *__restrict__ Bt, uint16_t *__restrict__ Bts,
+                               uint16_t *__restrict__ G, uint16_t *__restrict__ Bt, float *__restrict__ Bts,
                                int *status)
 {
     const int64_t nG = (int64_t)R1p * Kp, nB = Np * rp;
@@ -111,11 +111,10 @@ __global__ void pack_ec_kernel(const uint16_t *__restrict__ A, const uint16_t *_
             const uint16_t b = (n < N && j < r) ? B[j * N + n] : (uint16_t)0;
             Bt[e] = b;
             const float sn = s[n];
-            const float q = __fdiv_rn(__uint_as_float((uint32_t)b << 16), sn != 0.0f ? sn : 1.0f);
-            const __nv_bfloat16 qb = __float2bfloat16_rn(q);
-            if (!isfinite(__bfloat162float(qb)))
+            const float q = to_tf32(__fdiv_rn(__uint_as_float((uint32_t)b << 16), sn != 0.0f ? sn : 1.0f));
+            if (!isfinite(q))
                 atomicOr(status, kStatusNonFinite);
-            Bts[e] = __bfloat16_as_ushort(qb);
+            Bts[e] = q;
         }
     }
 }

@@ -4,7 +4,7 @@
 // Efficient Low-Bit LLM Serving", Abstract: the EC is "modulated by
 // per-token gates".  This library's reading of that gate and of the EC:
 //   logit_t = x[t,:] . w_g + b_g,   g_t = 1 / (1 + exp(-logit_t))
-//   u[t,j]  = x[t,:] . A[:,j]       v[t,j] = bf16(g_t * u[t,j])
+//   u[t,j]  = x[t,:] . A[:,j]       v[t,j] = g_t * u[t,j]   (fp32)
 // v is the left operand of the EC up-projection that the GEMM kernels add
 // to their accumulators (y += v . B).
 //
@@ -32,8 +32,8 @@ struct PrepassParams {
     float b_g;
     int S;       // CTAs per token tile (split-K)
     int bps;     // 64-wide k blocks per split
-    uint16_t *v;
-    float *vf;
+    float *v;
+    int tf32;
     float *g;
     float *part;
     unsigned *counters;
@@ -153,9 +153,7 @@ __global__ void __launch_bounds__(128) prepass_kernel(PrepassParams p)
         if (t >= p.M)
             continue;
         const float val = (j < p.r) ? s_gate[tt] * red[(1 + j) * kTok + tt] : 0.f;
-        p.v[t * p.rp + j] = __bfloat16_as_ushort(__float2bfloat16_rn(val));
-        if (p.vf)
-            p.vf[t * p.rp + j] = val;
+        p.v[t * p.rp + j] = p.tf32 ? to_tf32(val) : val;
     }
 }
 
@@ -204,7 +202,7 @@ size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms)
 
 int prepass_counters(int64_t max_M) { return (int)((max_M + kTok - 1) / kTok); }
 
-cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t *v, float *vf, float *g,
+cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
                            const PrepassWork &w, cudaStream_t st, int num_sms)
 {
     if (M <= 0 || pk.r == 0)
@@ -224,7 +222,7 @@ cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, uint16_t 
     p.bps = (nkb + p.S - 1) / p.S;
     p.S = (nkb + p.bps - 1) / p.bps;  // drop empty splits
     p.v = v;
-    p.vf = vf;
+    p.tf32 = tf32 ? 1 : 0;
     p.g = g;
     p.part = w.part;
     p.counters = w.counters;

@@ -25,8 +25,7 @@ struct spear_w4ec {
     Packed pk{};
     bool packed = false;
     // workspace
-    uint16_t *v = nullptr;      // [max_M][rp] bf16: g_t * (x . A)
-    float *vf = nullptr;        // the same in fp32 (split path)
+    float *v = nullptr;         // [max_M][rp] fp32: g_t * (x . A) (tf32-rounded for the tcgen05 path)
     float *gbuf = nullptr;      // [max_M] gate values
     PrepassWork pre{};
     DecodeWork dec{};
@@ -108,7 +107,6 @@ void free_all(spear_w4ec *h)
     cudaFree(h->pk.Bt);
     cudaFree(h->pk.Bts);
     cudaFree(h->v);
-    cudaFree(h->vf);
     cudaFree(h->gbuf);
     cudaFree(h->pre.part);
     cudaFree(h->pre.counters);
@@ -152,6 +150,15 @@ uint32_t resolve(const spear_w4ec *h, int64_t M, uint32_t flags)
     return path | mode;
 }
 
+// Gate and v for M tokens: the tcgen05 kernel from 256 tokens on, the
+// split-K mma.sync kernel below that.
+cudaError_t run_prepass(const spear_w4ec *h, const void *x, int64_t M, bool tf32, cudaStream_t st)
+{
+    if (M >= 256 && tc_prepass_supported(h->pk))
+        return launch_tc_prepass(h->pk, x, M, h->v, tf32, h->gbuf, h->tc, h->status, st);
+    return launch_prepass(h->pk, x, M, h->v, tf32, h->gbuf, h->pre, st, h->num_sms);
+}
+
 int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t flags, cudaStream_t st)
 {
     const Packed &pk = h->pk;
@@ -170,7 +177,7 @@ int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t
         return SPEAR_ERR_UNSUPPORTED;
     // the decode kernel computes its own gate and EC down-projection when fused
     if (ec && !(decode && fused)) {
-        e = launch_prepass(pk, x, M, h->v, fused ? nullptr : h->vf, h->gbuf, h->pre, st, h->num_sms);
+        e = run_prepass(h, x, M, (choice & SPEAR_FORCE_TC) != 0 && fused, st);
         if (e != cudaSuccess)
             return from_cuda(e);
     }
@@ -191,7 +198,7 @@ int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t
         }
     }
     if (ec && !fused) {
-        e = launch_ec_apply(pk, h->vf, y, M, st);
+        e = launch_ec_apply(pk, h->v, y, M, st);
         if (e != cudaSuccess)
             return from_cuda(e);
     }
@@ -268,7 +275,6 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r, const s
         chk(alloc_zero(&pk.Bt, (size_t)pk.Np * pk.rp));
         chk(alloc_zero(&pk.Bts, (size_t)pk.Np * pk.rp));
         chk(alloc_zero(&h->v, (size_t)h->max_M * pk.rp));
-        chk(alloc_zero(&h->vf, (size_t)h->max_M * pk.rp));
         chk(alloc_zero(&h->gbuf, (size_t)h->max_M));
         h->pre.part_floats = prepass_part_floats(pk, h->max_M, h->num_sms);
         h->pre.n_counters = prepass_counters(h->max_M);
@@ -412,7 +418,7 @@ int spear_w4ec_get_gate(const spear_w4ec *h, const void *x, float *g, int64_t M,
         return SPEAR_OK;
     DeviceGuard guard(h->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_prepass(h->pk, x, M, h->v, nullptr, h->gbuf, h->pre, st, h->num_sms);
+    cudaError_t e = run_prepass(h, x, M, false, st);
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(g, h->gbuf, (size_t)M * sizeof(float), cudaMemcpyDeviceToDevice, st);
     return from_cuda(e);

@@ -5,25 +5,27 @@
 // SPEAR, "A System for Post-Quantization Error-Adaptive Recovery Enabling
 // Efficient Low-Bit LLM Serving", Abstract: the post-EC computation is fused
 // into the low-bit GEMM.  Here the EC is literally part of the same
-// accumulation: after the K loop of the main product the tile runs r/16 more
-// MMA k-steps with v = g * (x . A) (from the prepass) against B^T, into the
-// same TMEM accumulator, so
+// accumulation: after the K loop of the main product the tile runs r/8 more
+// MMA k-steps, in tf32 (fp32 range, 2^-11 rounding: the EC operands v and
+// B^T/s need both), with v = g * (x . A) (from the prepass) against B^T/s,
+// into the same TMEM accumulator, so
 //     D[n, t] = sum_k (q[n,k] - z[n]) x[t,k] + sum_j (B[j,n] / s[n]) v[t,j]
 // and the epilogue writes y[t, n] = bf16(s[n] * D[n, t]).
 //
-// Layout of one CTA (persistent, one per SM, 10 warps):
+// Layout of one CTA (persistent, one per SM, 14 warps):
 //   warp 0      TMA producer: x tile (256 tokens x 64 k, 128B-swizzled) and
 //               the int4 code tile (128 rows x 64 k) per stage; for the EC
-//               stages the B^T tile and the v tile instead.
+//               stages the B^T/s tile and the v tile (32 fp32 j each) instead.
 //   warp 1      TMEM allocator and the single MMA-issuing thread:
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128 weight rows,
 //               N = 256 tokens, K = 16 per instruction (swap-AB: weights
 //               on the M side so one dequantised tile serves 256 tokens).
-//   warps 2-5   dequantisers: thread i owns weight row i of the tile and
-//               writes the exact integers (q - z) as bf16 into the
-//               128B-swizzled K-major A tile of the stage (the layout the
-//               MMA descriptor names).
-//   warps 6-9   epilogue: tcgen05.ld of the finished accumulator (each warp
+//   warps 2-9   dequantisers: thread (i, h) owns half h of weight row i of
+//               the tile (32 k) and writes the exact integers (q - z) as
+//               bf16 into the 128B-swizzled K-major A tile of the stage (the
+//               layout the MMA descriptor names); two warps per SM sub-
+//               partition so one hides the other's latency.
+//   warps 10-13 epilogue: tcgen05.ld of the finished accumulator (each warp
 //               its 32-lane quarter), times the channel scale s[n], bf16
 //               rounding, stores of y[t, n].
 // The accumulator holds sum_k x (q - z) exactly up to fp32 summation, so the
@@ -31,7 +33,7 @@
 // s[n] in the epilogue scales both terms.
 // Four stages of 52 KB in shared memory; two 256-column accumulators in
 // TMEM so the epilogue of one tile overlaps the main loop of the next.
-// Every mbarrier wait is bounded (about a second of %globaltimer); a wait
+// Every mbarrier wait is bounded (about a second of SM clock cycles); a wait
 // that runs out sets the handle's status word and the kernel winds down.
 #include <new>
 
@@ -51,7 +53,7 @@ constexpr int B_BYTES = BN * BK * 2;          // 32 KB activations (or v on EC s
 constexpr int C_BYTES = BM * BK / 2;          // 4 KB int4 codes
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-constexpr int THREADS = 320;
+constexpr int THREADS = 448;   // 14 warps: TMA, MMA, 8 dequantisers, 4 epilogue
 constexpr int TMEM_COLS = 2 * BN;
 
 struct TcParams {
@@ -68,7 +70,156 @@ struct TcParams {
 struct Maps {
     CUtensorMap codes;
     CUtensorMap bt;
+    CUtensorMap g;   // G = [w_g; A^T] [R1p][Kp] bf16, boxes of 64 x R1p, 128B swizzle
 };
+
+// ---------------------------------------------------------------- EC down-projection for many tokens
+//
+// D[t, j] = x[t, :] . G[j, :] for a 128-token tile, G = [w_g; A^T] (R1p <= 256
+// rows): tcgen05.mma with the tokens on the M = 128 side (TMEM lanes) and the
+// R1p rows of G on N, so each epilogue thread owns one token's whole row of D
+// and forms g_t = sigmoid(D[t,0] + b_g) and v[t, j] = g_t * D[t, 1+j] alone.
+// Warp 0: TMA producer; warp 1: TMEM allocator and MMA issuer; warps 2-5:
+// epilogue.  One tile per CTA, 4 stages of x (16 KB) and G (R1p x 128 B).
+
+constexpr int PP_STAGES = 4;
+constexpr int PP_THREADS = 192;
+
+struct PrepassTcParams {
+    int64_t M;
+    int n_k;            // 64-wide k stages
+    int R1p, r, rp;
+    float b_g;
+    float *v;           // [M][rp] fp32
+    int tf32;           // round v to tf32
+    float *g;           // [M]
+    int *status;
+};
+
+__global__ void __launch_bounds__(PP_THREADS, 1)
+tc_prepass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_g,
+                  PrepassTcParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t bars[2 * PP_STAGES + 2];
+    __shared__ uint32_t tmem_base_slot;
+    __shared__ volatile int abort_flag;
+
+    pdl_launch_dependents();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+    const uint32_t x_bytes = 128 * 128, g_bytes = (uint32_t)p.R1p * 128;
+    const uint32_t stage_bytes = x_bytes + ((g_bytes + 1023u) & ~1023u);
+    const uint32_t full0 = smem_addr(&bars[0]), empty0 = smem_addr(&bars[PP_STAGES]);
+    const uint32_t done = smem_addr(&bars[2 * PP_STAGES]), drain = smem_addr(&bars[2 * PP_STAGES + 1]);
+    const int t0 = blockIdx.x * 128;
+    uint32_t tmem_cols = 32;
+    while (tmem_cols < (uint32_t)p.R1p)
+        tmem_cols <<= 1;
+
+    if (tid == 0) {
+        abort_flag = 0;
+        for (int s = 0; s < PP_STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(done, 1);
+        mbar_init(drain, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&tmem_base_slot)),
+                     "r"(tmem_cols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            pdl_wait();  // x comes from an earlier kernel in the stream
+            int issued = 0;
+            for (int kb = 0; kb < p.n_k; ++kb, ++issued) {
+                const uint32_t slot = kb % PP_STAGES, phase = (kb / PP_STAGES) & 1;
+                if (!mbar_wait(empty0 + 8 * slot, phase ^ 1, &abort_flag, p.status))
+                    break;
+                const uint32_t sb = base + slot * stage_bytes;
+                mbar_expect_tx(full0 + 8 * slot, x_bytes + g_bytes);
+                tma_load_2d(sb, &tm_x, kb * 64, t0, full0 + 8 * slot);
+                tma_load_2d(sb + x_bytes, &tm_g, kb * 64, 0, full0 + 8 * slot);
+            }
+            for (int k = 0; k < PP_STAGES && k < issued; ++k) {
+                const int kb = issued - 1 - k;
+                mbar_wait_final(full0 + 8 * (kb % PP_STAGES), (kb / PP_STAGES) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(p.R1p >> 3) << 17) |
+                                   ((uint32_t)(128 >> 4) << 24);
+            bool ok = true;
+            for (int kb = 0; kb < p.n_k && ok; ++kb) {
+                const uint32_t slot = kb % PP_STAGES, phase = (kb / PP_STAGES) & 1;
+                if (!mbar_wait(full0 + 8 * slot, phase, &abort_flag, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sb = base + slot * stage_bytes;
+                const uint64_t a_desc = smem_desc_sw128(sb), b_desc = smem_desc_sw128(sb + x_bytes);
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16(tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (kb > 0 || k > 0) ? 1u : 0u);
+                mma_commit(empty0 + 8 * slot);
+            }
+            if (ok)
+                mma_commit(done);
+            // every MMA of this thread is complete before TMEM is released
+            mma_commit(drain);
+            mbar_wait_final(drain, 0);
+        }
+    } else {
+        // epilogue: warp (2..5) & 3 owns TMEM lanes 32q..32q+31 = tokens
+        const int q = warp & 3;
+        const int64_t t = t0 + 32 * q + lane;
+        if (mbar_wait(done, 0, &abort_flag, p.status)) {
+            tc_fence_after();
+            float gt = 0.f;
+            for (int c = 0; c < p.R1p; c += 32) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + c, r);
+                if (c == 0)
+                    gt = 1.0f / (1.0f + expf(-(__uint_as_float(r[0]) + p.b_g)));
+                if (t < p.M) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int j = c + i - 1;   // column c+i holds x . A[:, c+i-1]
+                        if (j >= 0 && j < p.rp) {
+                            const float val = j < p.r ? gt * __uint_as_float(r[i]) : 0.f;
+                            p.v[t * p.rp + j] = p.tf32 ? to_tf32(val) : val;
+                        }
+                    }
+                }
+            }
+            // v columns past the last column of D (only when r + 1 fills R1p exactly) are zero
+            if (t < p.M)
+                for (int j = p.R1p - 1; j < p.rp; ++j)
+                    p.v[t * p.rp + j] = 0.f;
+            if (t < p.M)
+                p.g[t] = gt;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols) : "memory");
+    }
+}
 
 // ---------------------------------------------------------------- the kernel
 
@@ -96,7 +247,7 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         abort_flag = 0;
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(full0 + 8 * s, 1);
-            mbar_init(aready0 + 8 * s, 128);
+            mbar_init(aready0 + 8 * s, 256);
             mbar_init(empty0 + 8 * s, 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -143,10 +294,10 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         tma_load_4d(sb + A_BYTES + B_BYTES + C_BYTES / 2, &tm_codes, 0, st & 3, 0, blk + p.kchunks,
                                     full);
                     } else {
-                        const int e = st - p.n_main;
+                        const int e = st - p.n_main;   // 32 tf32 values of j per EC stage
                         mbar_expect_tx(full, A_BYTES + B_BYTES);
-                        tma_load_2d(sb, &tm_bt, e * BK, n0, full);
-                        tma_load_2d(sb + A_BYTES, &tm_v, e * BK, t0, full);
+                        tma_load_2d(sb, &tm_bt, e * 32, n0, full);
+                        tma_load_2d(sb + A_BYTES, &tm_v, e * 32, t0, full);
                     }
                 }
             }
@@ -163,6 +314,10 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                                    | (1u << 7) | (1u << 10)     // A, B: bf16
                                    | ((uint32_t)(BN >> 3) << 17)
                                    | ((uint32_t)(BM >> 4) << 24);
+            const uint32_t idesc_tf32 = (1u << 4)               // D: f32
+                                        | (2u << 7) | (2u << 10)  // A, B: tf32
+                                        | ((uint32_t)(BN >> 3) << 17)
+                                        | ((uint32_t)(BM >> 4) << 24);
             uint32_t g = 0;
             int lt = 0;
             bool ok = true;
@@ -182,13 +337,16 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     tc_fence_after();
                     const uint32_t sb = base + slot * STAGE_BYTES;
                     const uint64_t a_desc = smem_desc_sw128(sb), b_desc = smem_desc_sw128(sb + A_BYTES);
-                    int ksteps = BK / 16;
-                    if (st >= p.n_main) {
-                        const int rem = p.rp - (st - p.n_main) * BK;
-                        ksteps = (rem < BK ? rem : BK) / 16;
+                    if (st < p.n_main) {
+                        for (int k = 0; k < BK / 16; ++k)
+                            mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (st > 0 || k > 0) ? 1u : 0u);
+                    } else {
+                        // EC: 32 tf32 values of j per 128-byte row, 8 per instruction
+                        const int rem = p.rp - (st - p.n_main) * 32;
+                        const int ksteps = (rem < 32 ? rem : 32) / 8;
+                        for (int k = 0; k < ksteps; ++k)
+                            mma_tf32(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc_tf32, 1u);
                     }
-                    for (int k = 0; k < ksteps; ++k)
-                        mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (st > 0 || k > 0) ? 1u : 0u);
                     mma_commit(empty0 + 8 * slot);
                 }
                 if (ok)
@@ -198,9 +356,9 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             mma_commit(drain);
             mbar_wait_final(drain, 0);
         }
-    } else if (warp < 6) {
-        // ------------------------------------------------ dequantisers: thread i = weight row i
-        const int i = tid - 64;
+    } else if (warp < 10) {
+        // ------------------------------------------------ dequantisers: thread (i, h) = half h of weight row i
+        const int i = (tid - 64) & 127, half = (tid - 64) >> 7;
         uint32_t g = 0;
         for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
             const int n = (tile / p.n_ttiles) * BM + i;
@@ -215,15 +373,18 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 }
                 if (st < p.n_main) {
                     uint8_t *sb = base_ptr + slot * STAGE_BYTES;
-                    const uint4 *cw = reinterpret_cast<const uint4 *>(sb + A_BYTES + B_BYTES + i * 32);
-                    const uint4 w0 = cw[0], w1 = cw[1];
-                    const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                    // code row i: 32 bytes (64 k), its two 16-byte halves swapped in rows
+                    // with bit 2 set (32-byte TMA swizzle, conflict-free reads)
+                    const uint4 w0 = *reinterpret_cast<const uint4 *>(sb + A_BYTES + B_BYTES + i * 32 +
+                                                                      ((half ^ ((i >> 2) & 1)) << 4));
+                    const uint32_t words[4] = {w0.x, w0.y, w0.z, w0.w};
                     uint8_t *arow = sb + i * 128;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
+                    for (int jj = 0; jj < 4; ++jj) {
+                        const int j = 4 * half + jj;
                         // codes k = 8j + {0..7}: pairs (0,4) (1,5) (2,6) (3,7)
-                        const uint32_t p0 = dequant_pair(words[j], negz), p1 = dequant_pair(words[j] >> 4, negz);
-                        const uint32_t p2 = dequant_pair(words[j] >> 8, negz), p3 = dequant_pair(words[j] >> 12, negz);
+                        const uint32_t p0 = dequant_pair(words[jj], negz), p1 = dequant_pair(words[jj] >> 4, negz);
+                        const uint32_t p2 = dequant_pair(words[jj] >> 8, negz), p3 = dequant_pair(words[jj] >> 12, negz);
                         uint4 o;
                         o.x = prmt(p0, p1, 0x5410);   // k 0, 1
                         o.y = prmt(p2, p3, 0x5410);   // k 2, 3
@@ -306,14 +467,17 @@ cudaError_t tc_prepare(const Packed &pk, TcWork &w)
     const uint64_t strides[3] = {32, 128, 8192};
     const uint32_t box[4] = {8, 1, 64, 1};
     cudaError_t e = make_map_nd(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, dims, strides, box,
-                                CU_TENSOR_MAP_SWIZZLE_NONE);
+                                CU_TENSOR_MAP_SWIZZLE_32B);
     if (e == cudaSuccess && pk.r > 0)
-        e = make_map(&m->bt, pk.Bts, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.rp, (uint64_t)pk.Np, BK, BM,
+        e = make_map(&m->g, pk.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.Kp, (uint64_t)pk.R1p, 64,
+                     (uint32_t)pk.R1p, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e == cudaSuccess && pk.r > 0)
+        e = make_map(&m->bt, pk.Bts, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)pk.rp, (uint64_t)pk.Np, 32, BM,
                      CU_TENSOR_MAP_SWIZZLE_128B);
     return e;
 }
 
-cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const uint16_t *v, bool ec,
+cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const float *v, bool ec,
                       const TcWork &w, int *status, bool zero_wait_budget, cudaStream_t st, int num_sms)
 {
     if (M <= 0)
@@ -333,7 +497,7 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
         return e;
     const bool use_ec = ec && pk.r > 0;
     if (use_ec) {
-        e = make_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.rp, (uint64_t)M, BK, BN,
+        e = make_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)pk.rp, (uint64_t)M, 32, BN,
                      CU_TENSOR_MAP_SWIZZLE_128B);
         if (e != cudaSuccess)
             return e;
@@ -345,7 +509,7 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
     p.N = pk.N;
     p.kchunks = (int)(pk.Kp / 256);
     p.n_main = (int)(pk.Kp / BK);
-    p.n_ec = use_ec ? (pk.rp + BK - 1) / BK : 0;
+    p.n_ec = use_ec ? (pk.rp + 31) / 32 : 0;   // 32 tf32 values per 128-byte row
     p.rp = pk.rp;
     p.n_ttiles = (int)((M + BN - 1) / BN);
     p.n_tiles = p.n_ttiles * (int)(pk.Np / BM);
@@ -368,6 +532,54 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, tc_w4ec_kernel, tm_x, m->codes, use_ec ? m->bt : m->codes, tm_v, p);
+}
+
+}  // namespace spear
+
+namespace spear {
+
+bool tc_prepass_supported(const Packed &pk) { return pk.r > 0 && pk.R1p <= 256 && tensor_maps_available(); }
+
+cudaError_t launch_tc_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
+                              const TcWork &w, int *status, cudaStream_t st)
+{
+    if (M <= 0)
+        return cudaSuccess;
+    const Maps *m = static_cast<const Maps *>(w.maps);
+    if (!m || !tc_prepass_supported(pk))
+        return cudaErrorInvalidValue;
+    CUtensorMap tm_x;
+    cudaError_t e = make_map(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.K, (uint64_t)M, 64, 128,
+                             CU_TENSOR_MAP_SWIZZLE_128B);
+    if (e != cudaSuccess)
+        return e;
+    PrepassTcParams p;
+    p.M = M;
+    p.n_k = (int)(pk.Kp / 64);
+    p.R1p = pk.R1p;
+    p.r = pk.r;
+    p.rp = pk.rp;
+    p.b_g = pk.b_g;
+    p.v = v;
+    p.tf32 = tf32 ? 1 : 0;
+    p.g = g;
+    p.status = status;
+    const uint32_t stage = 128 * 128 + (((uint32_t)pk.R1p * 128 + 1023u) & ~1023u);
+    const size_t smem = (size_t)PP_STAGES * stage + 1024;
+    e = raise_smem_limit(reinterpret_cast<const void *>(tc_prepass_kernel), smem);
+    if (e != cudaSuccess)
+        return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((M + 127) / 128));
+    cfg.blockDim = dim3(PP_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, tc_prepass_kernel, tm_x, m->g, p);
 }
 
 }  // namespace spear
