@@ -152,12 +152,13 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 
     bool ok = wait_bounded(bar_x, 0);
 
-    float acc[T][4];
+    // two accumulator sets (even / odd code word) halve the MMA dependency chains
+    float acc[T][4], acc2[T][4];
 #pragma unroll
     for (int n = 0; n < T; ++n)
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            acc[n][i] = 0.f;
+            acc[n][i] = acc2[n][i] = 0.f;
 
     float *red = reinterpret_cast<float *>(bp + L.red);
     if (!is_u) {
@@ -197,12 +198,18 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 #pragma unroll
                     for (int n = 0; n < T; ++n) {
                         const uint4 v = xv[n][j];
-                        mma_bf16_16816(acc[n], g0, h0, g1, h1, prmt(v.x, v.z, 0x5410), prmt(v.x, v.z, 0x7632));
-                        mma_bf16_16816(acc[n], g2, h2, g3, h3, prmt(v.y, v.w, 0x5410), prmt(v.y, v.w, 0x7632));
+                        float (&a)[4] = j ? acc2[n] : acc[n];
+                        mma_bf16_16816(a, g0, h0, g1, h1, prmt(v.x, v.z, 0x5410), prmt(v.x, v.z, 0x7632));
+                        mma_bf16_16816(a, g2, h2, g3, h3, prmt(v.y, v.w, 0x5410), prmt(v.y, v.w, 0x7632));
                     }
                 }
             }
         }
+#pragma unroll
+        for (int n = 0; n < T; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                acc[n][i] += acc2[n][i];
         float *mine = red + kpar * kRows * TOK;   // [2][64][TOK]
 #pragma unroll
         for (int n = 0; n < T; ++n) {
@@ -237,10 +244,15 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 // natural pairs: step s covers k = 16 cl + 4s + {0,1} and + {2,3}
 #pragma unroll
                 for (int s = 0; s < 4; ++s)
-                    mma_bf16_16816(acc[n], ga[2 * s], ha[2 * s], ga[2 * s + 1], ha[2 * s + 1], xa[2 * s],
-                                   xa[2 * s + 1]);
+                    mma_bf16_16816((s & 1) ? acc2[n] : acc[n], ga[2 * s], ha[2 * s], ga[2 * s + 1], ha[2 * s + 1],
+                                   xa[2 * s], xa[2 * s + 1]);
             }
         }
+#pragma unroll
+        for (int n = 0; n < T; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                acc[n][i] += acc2[n][i];
         float *mine = red + warp * 16 * TOK;  // [8 warps][16][TOK]
 #pragma unroll
         for (int n = 0; n < T; ++n) {
@@ -387,19 +399,35 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     }
 }
 
+// Cluster size CS (CTAs splitting K) and the k per CTA, or 0 if a slice would
+// not fit in shared memory.  Preferably the grid takes about two CTAs per SM,
+// so that the next layer's kernel (launched early) finds room to start its
+// weight copies while this one runs; layers too large for that take up to 8
+// CTAs per SM.  No rank is left without a chunk.
 int pick_cluster(const Packed &pk, int num_sms, int JB, int *KS_out)
 {
     const int NC = (int)(pk.Np / kRows);
     const int chunks = (int)(pk.Kp / kChunk);
-    int CS = std::min(8, chunks);
-    // no more than about 8 CTAs per SM, and no rank left without a chunk
-    while (CS > 1 && ((int64_t)(NC + JB) * CS > 8LL * num_sms || (CS - 1) * ((chunks + CS - 1) / CS) >= chunks))
-        --CS;
-    const int per = (chunks + CS - 1) / CS;
-    if (per > kMaxChunks)
-        return 0;
-    *KS_out = per * kChunk;
-    return CS;
+    for (int limit : {2, 8}) {
+        for (int CS = std::min(8, chunks); CS >= 1; --CS) {
+            const int per = (chunks + CS - 1) / CS;
+            if (per > kMaxChunks || (CS - 1) * per >= chunks)
+                continue;
+            if ((int64_t)(NC + JB) * CS <= (int64_t)limit * num_sms) {
+                *KS_out = per * kChunk;
+                return CS;
+            }
+        }
+    }
+    // otherwise the fewest chunks per CTA that fit
+    for (int CS = std::min(8, chunks); CS >= 1; --CS) {
+        const int per = (chunks + CS - 1) / CS;
+        if (per <= kMaxChunks && (CS == 1 || (CS - 1) * per < chunks)) {
+            *KS_out = per * kChunk;
+            return CS;
+        }
+    }
+    return 0;
 }
 
 template <int T>

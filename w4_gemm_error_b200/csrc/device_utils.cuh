@@ -42,11 +42,12 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t w_shifted, uint32_t ne
     return fma_bf16x2(t, 0x3F803F80u /* (1.0, 1.0) */, neg_bias);
 }
 
-// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col).
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col).  Not volatile: its
+// only effect is on d, so the compiler may interleave independent MMAs.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1)
 {
-    asm volatile(
+    asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
