@@ -22,8 +22,13 @@
 //    nibbles 16 bits apart per register), and the activations are paired to
 //    match with one byte permute per register, the k order inside the MMA
 //    being permuted accordingly;
-//  * the K split is summed over distributed shared memory inside the
-//    cluster, in rank order (deterministic), with no global round trip;
+//  * the K split is summed inside the cluster, in rank order
+//    (deterministic), with no global round trip: the other CTAs push their
+//    partial tiles into receive slots of the first CTA (st.async, counted on
+//    one mbarrier whose cluster handshake happens before the wait for the
+//    previous kernel); where the slots do not fit in shared memory the first
+//    CTA pulls the tiles over distributed shared memory between two cluster
+//    barriers instead;
 //  * the EC down-projection u = x . [w_g, A] runs on R1p/16 extra clusters
 //    of the same grid (the first ones) with the same slicing; they publish u
 //    in global memory behind a counter, and the 64-row clusters read it for
@@ -65,16 +70,18 @@ struct DecodeParams {
     int KS, nch;          // k per CTA (a multiple of 256), code chunks per CTA
     int JB, NC;           // EC clusters, 64-row clusters
     int r, rp, R1p;
+    int push;             // partial tiles pushed into receive slots of the first CTA
     float b_g;
 };
 
 struct Smem {
-    uint32_t codes, x, bt, red, u;   // byte offsets from the 1024-aligned base
+    uint32_t codes, x, bt, red, u, recv;   // byte offsets from the 1024-aligned base
     uint32_t total;
 };
 
+// nslots receive slots of one partial tile (64 rows x TOK fp32) each.
 template <int TOK>
-__host__ __device__ inline Smem smem_layout(int KS, int rp, int R1p)
+__host__ __device__ inline Smem smem_layout(int KS, int rp, int R1p, int nslots)
 {
     Smem m;
     m.codes = 0;                                   // 32*KS bytes: codes (64 rows) or G (16 rows bf16)
@@ -82,13 +89,52 @@ __host__ __device__ inline Smem smem_layout(int KS, int rp, int R1p)
     m.bt = m.x + 2 * TOK * KS;                     // 128*rp bytes: B^T rows of the cluster
     m.red = m.bt + 128 * rp;                       // 512*TOK bytes: partial tiles
     m.u = m.red + 512 * TOK;                       // u [R1p][TOK], g [TOK], v [TOK][rp] (fp32)
-    m.total = m.u + 4 * R1p * TOK + 4 * TOK * (rp + 1);
+    m.recv = (m.u + 4 * R1p * TOK + 4 * TOK * (rp + 1) + 15) & ~15u;
+    m.total = m.recv + nslots * 256 * TOK;
     return m;
 }
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) { return mbar_wait_bounded(bar, parity); }
 
 constexpr int kThreads = 256;   // 8 warps: two per 16-row group, splitting the sub-blocks
+constexpr int kEcWarp = kThreads / 32 - 1;
+
+// One warp: wait (bounded) until the EC clusters have published u, copy u
+// [R1p][TOK] into shared memory, then g [TOK] and v [TOK][rp] = g * u[1..r].
+template <int TOK>
+__device__ __forceinline__ void fetch_u(const DecodeParams &p, float *us, float *gs, float *vv, int lane)
+{
+    int good = 1;
+    if (lane == 0) {
+        const long long t0 = clock64();
+        while (ld_acquire_gpu(&p.flags[0]) < (unsigned)p.JB) {
+            if (clock64() - t0 > kWaitBudgetCycles) {
+                atomicOr(p.status, kStatusTimeout);
+                good = 0;
+                break;
+            }
+            __nanosleep(32);
+        }
+    }
+    good = __shfl_sync(0xffffffffu, good, 0);
+    for (int e = lane; e < p.R1p * TOK; e += 32) {
+        const int row = e / TOK, t = e - row * TOK;
+        us[e] = good ? __ldcg(p.ws_u + row * kUStride + t) : 0.f;
+    }
+    __syncwarp();
+    if (lane == 0 && atomicAdd(&p.flags[1], 1u) == (unsigned)(p.NC - 1)) {
+        // every 64-row cluster has read u: reset for the next forward
+        p.flags[1] = 0u;
+        p.flags[0] = 0u;
+    }
+    for (int t = lane; t < TOK; t += 32)
+        gs[t] = 1.0f / (1.0f + expf(-(us[t] + p.b_g)));
+    __syncwarp();
+    for (int e = lane; e < TOK * p.rp; e += 32) {
+        const int t = e / p.rp, j = e - t * p.rp;
+        vv[e] = j < p.r ? gs[t] * us[(1 + j) * TOK + t] : 0.f;
+    }
+}
 
 template <int T>
 __global__ void __launch_bounds__(kThreads)
@@ -98,15 +144,15 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 {
     constexpr int TOK = 8 * T;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[kMaxChunks + 2];
-    __shared__ int s_ok;
+    __shared__ __align__(8) uint64_t bars[kMaxChunks + 3];
 
     pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, cl = lane & 3;
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const bp = smem_raw + (base - raw);
-    const Smem L = smem_layout<TOK>(p.KS, p.rp, p.R1p);
+    const bool push = p.push != 0;
+    const Smem L = smem_layout<TOK>(p.KS, p.rp, p.R1p, push ? CS - 1 : 0);
     const uint32_t rank = cluster_ctarank();
     const int cluster = blockIdx.x / CS;
     const bool is_u = cluster < p.JB;
@@ -117,14 +163,23 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     const uint32_t bar_chunk = smem_addr(&bars[0]);
     const uint32_t bar_x = smem_addr(&bars[kMaxChunks]);
     const uint32_t bar_bt = smem_addr(&bars[kMaxChunks + 1]);
+    const uint32_t bar_recv = smem_addr(&bars[kMaxChunks + 2]);
     const int n0 = is_u ? 0 : (cluster - p.JB) * kRows;
+    const int tile_rows = is_u ? 16 : kRows;
 
-    // epilogue scale of this thread's row, requested before anything else
+    // loads that do not depend on earlier kernels are issued before waiting
+    // for them: the epilogue scale of this thread's row and the zero points
+    // of its two MMA rows
     const float s_epi = (!is_u && rank == 0) ? __ldg(p.s + n0 + (tid & (kRows - 1))) : 0.f;
+    const int rg = 16 * (warp & 3) + gid;  // MMA rows rg and rg + 8 (64-row clusters)
+    const uint32_t zg_raw = is_u ? 0u : (uint32_t)__ldg(p.z + n0 + rg);
+    const uint32_t zh_raw = is_u ? 0u : (uint32_t)__ldg(p.z + n0 + rg + 8);
     if (tid == 0) {
-        for (int c = 0; c < kMaxChunks + 2; ++c)
+        for (int c = 0; c < kMaxChunks + 3; ++c)
             mbar_init(bar_chunk + 8 * c, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        fence_mbarrier_init_cluster();
+        if (push && rank == 0 && CS > 1)
+            mbar_expect_tx(bar_recv, (uint32_t)((CS - 1) * tile_rows * TOK * 4));
         // the weights do not depend on earlier kernels: start them now
         for (int c = 0; c < nch; ++c) {
             const uint32_t bar = bar_chunk + 8 * c;
@@ -142,13 +197,17 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             mbar_expect_tx(bar_bt, 128 * p.rp);   // B^T rows of the cluster, for the epilogue
             tma_load_2d(base + L.bt, &tm_bt, 0, n0, bar_bt);
         }
+    }
+    __syncthreads();
+    if (push)
+        cluster_arrive_relaxed();   // the receive barrier of the first CTA is initialised
+    if (tid == 0) {
         // the activations are written by the previous kernel in the stream
         pdl_wait();
         mbar_expect_tx(bar_x, 2 * TOK * kChunk * nch);
         for (int i = 0; i < nsub; ++i)
             tma_load_2d(base + L.x + i * (TOK * 128), &tm_x, k0 + 64 * i, 0, bar_x);
     }
-    __syncthreads();
 
     bool ok = wait_bounded(bar_x, 0);
 
@@ -163,11 +222,9 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     float *red = reinterpret_cast<float *>(bp + L.red);
     if (!is_u) {
         // ---- 64 weight rows: warps w and w+4 own rows 16w .. 16w+15, sub-blocks of parity w>>2
-        const int rg = 16 * (warp & 3) + gid;  // and rg + 8 (same row mod 8)
         const int kpar = warp >> 2;
-        const uint32_t zg = 128u + p.z[n0 + rg], zh = 128u + p.z[n0 + rg + 8];
-        const uint32_t nbg = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)zg));
-        const uint32_t nbh = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)zh));
+        const uint32_t nbg = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + zg_raw)));
+        const uint32_t nbh = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + zh_raw)));
         const uint32_t negg = nbg | (nbg << 16), negh = nbh | (nbh << 16);
         for (int c = 0; c < nch && ok; ++c) {
             ok = wait_bounded(bar_chunk + 8 * c, 0);
@@ -284,34 +341,78 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             wait_bounded(bar_bt, 0);
     }
 
-    // ---- sum the K split over the cluster, in rank order, in the first CTA
-    __syncthreads();
-    cluster_sync();
-    const int tile = (is_u ? 16 : kRows) * TOK;
-    if (rank == 0) {
-        const uint32_t red_addr = base + L.red;
-        for (int e4 = tid; e4 < tile / 4; e4 += kThreads) {
-            // issue every remote load before summing (in rank order)
-            float4 o[8];
-#pragma unroll
-            for (int q = 1; q < 8; ++q)
-                if (q < CS)
-                    o[q] = ld_dsmem_f4(map_to_rank(red_addr + 16 * e4, (uint32_t)q));
-            float4 s = reinterpret_cast<const float4 *>(red)[e4];
-#pragma unroll
-            for (int q = 1; q < 8; ++q)
-                if (q < CS) {
-                    s.x += o[q].x;
-                    s.y += o[q].y;
-                    s.z += o[q].z;
-                    s.w += o[q].w;
-                }
-            reinterpret_cast<float4 *>(red)[e4] = s;
+    // ---- sum the K split over the cluster, in rank order, in the first CTA.
+    // In the first CTA of a 64-row cluster with an EC, the last warp fetches u
+    // meanwhile.
+    float *us = reinterpret_cast<float *>(bp + L.u);   // u [R1p][TOK]
+    float *gs = us + p.R1p * TOK;                      // g [TOK]
+    float *vv = gs + TOK;                              // v [TOK][rp] = g * u
+    const bool ec_warp = !is_u && rank == 0 && p.JB > 0 && warp == kEcWarp;
+    const int nsum = (!is_u && p.JB > 0) ? kThreads - 32 : kThreads;
+    const int tile4 = tile_rows * TOK / 4;
+    if (push) {
+        cluster_wait();   // every receive barrier of the cluster is initialised
+        if (rank != 0) {
+            const uint32_t dst = map_to_rank(base + L.recv + (rank - 1) * (tile_rows * TOK * 4), 0);
+            const uint32_t rbar = map_to_rank(bar_recv, 0);
+            for (int e4 = tid; e4 < tile4; e4 += kThreads)
+                st_async_f4(dst + 16 * e4, reinterpret_cast<const float4 *>(red)[e4], rbar);
+            cluster_arrive();
+            cluster_wait();   // the first CTA has received every tile
+            return;
         }
+        if (ec_warp) {
+            fetch_u<TOK>(p, us, gs, vv, lane);
+        } else if (CS > 1) {
+            if (!wait_bounded(bar_recv, 0) && tid == 0)
+                atomicOr(p.status, kStatusTimeout);
+        }
+        cluster_arrive();     // the tiles have landed: the other CTAs may leave
+        const float4 *slots = reinterpret_cast<const float4 *>(bp + L.recv);
+        if (!ec_warp)
+            for (int e4 = tid; e4 < tile4; e4 += nsum) {
+                float4 s = reinterpret_cast<const float4 *>(red)[e4];
+                for (int q = 0; q < CS - 1; ++q) {
+                    const float4 o = slots[q * tile4 + e4];
+                    s.x += o.x;
+                    s.y += o.y;
+                    s.z += o.z;
+                    s.w += o.w;
+                }
+                reinterpret_cast<float4 *>(red)[e4] = s;
+            }
+    } else {
+        __syncthreads();
+        cluster_sync();
+        if (rank == 0) {
+            if (ec_warp) {
+                fetch_u<TOK>(p, us, gs, vv, lane);
+            } else {
+                const uint32_t red_addr = base + L.red;
+                for (int e4 = tid; e4 < tile4; e4 += nsum) {
+                    // issue every remote load before summing (in rank order)
+                    float4 o[8];
+#pragma unroll
+                    for (int q = 1; q < 8; ++q)
+                        if (q < CS)
+                            o[q] = ld_dsmem_f4(map_to_rank(red_addr + 16 * e4, (uint32_t)q));
+                    float4 s = reinterpret_cast<const float4 *>(red)[e4];
+#pragma unroll
+                    for (int q = 1; q < 8; ++q)
+                        if (q < CS) {
+                            s.x += o[q].x;
+                            s.y += o[q].y;
+                            s.z += o[q].z;
+                            s.w += o[q].w;
+                        }
+                    reinterpret_cast<float4 *>(red)[e4] = s;
+                }
+            }
+        }
+        cluster_sync();  // the other CTAs' shared memory is no longer read
+        if (rank != 0)
+            return;
     }
-    cluster_sync();  // the other CTAs' shared memory is no longer read
-    if (rank != 0)
-        return;
     __syncthreads();
 
     if (is_u) {
@@ -324,50 +425,14 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         __syncthreads();
         if (tid == 0)
             atomicAdd(&p.flags[0], 1u);
+        if (push)
+            cluster_wait();
         return;
     }
 
     // ---- epilogue of a 64-row cluster
-    float *us = reinterpret_cast<float *>(bp + L.u);   // u [R1p][TOK]
-    float *gs = us + p.R1p * TOK;                      // g [TOK]
-    float *vv = gs + TOK;                              // v [TOK][rp] = g * u
-    if (p.JB > 0) {
-        if (tid == 0) {
-            int good = 1;
-            const long long t0 = clock64();
-            while (ld_acquire_gpu(&p.flags[0]) < (unsigned)p.JB) {
-                if (clock64() - t0 > kWaitBudgetCycles) {
-                    atomicOr(p.status, kStatusTimeout);
-                    good = 0;
-                    break;
-                }
-                __nanosleep(64);
-            }
-            s_ok = good;
-        }
-        __syncthreads();
-        for (int e = tid; e < p.R1p * TOK; e += kThreads) {
-            const int row = e / TOK, t = e - row * TOK;
-            us[e] = s_ok ? __ldcg(p.ws_u + row * kUStride + t) : 0.f;
-        }
-        __syncthreads();
-        if (tid == 0 && atomicAdd(&p.flags[1], 1u) == (unsigned)(p.NC - 1)) {
-            // every 64-row cluster has read u: reset for the next forward
-            p.flags[1] = 0u;
-            p.flags[0] = 0u;
-        }
-        if (tid < TOK)
-            gs[tid] = 1.0f / (1.0f + expf(-(us[tid] + p.b_g)));
-        __syncthreads();
-        for (int e = tid; e < TOK * p.rp; e += kThreads) {
-            const int t = e / p.rp, j = e - t * p.rp;
-            vv[e] = j < p.r ? gs[t] * us[(1 + j) * TOK + t] : 0.f;
-        }
-        if (!wait_bounded(bar_bt, 0))
-            atomicOr(p.status, kStatusTimeout);
-        __syncthreads();
-    }
-
+    if (p.JB > 0 && !wait_bounded(bar_bt, 0))
+        atomicOr(p.status, kStatusTimeout);
     const int row = tid & (kRows - 1), th = tid >> 6;  // four token phases
     const int64_t n = n0 + row;
     float out[TOK / 4];
@@ -397,6 +462,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         if (t < p.M && n < p.N)
             p.y[(int64_t)t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
     }
+    if (push)
+        cluster_wait();
 }
 
 // Cluster size CS (CTAs splitting K) and the k per CTA, or 0 if a slice would
@@ -446,7 +513,7 @@ bool decode_supported(const Packed &pk, int num_sms)
     const int CS = pick_cluster(pk, num_sms, pk.r > 0 ? pk.R1p / 16 : 0, &KS);
     if (CS == 0)
         return false;
-    return smem_layout<32>(KS, pk.rp, pk.R1p).total + 1024 <= 227 * 1024;
+    return smem_layout<32>(KS, pk.rp, pk.R1p, 0).total + 1024 <= 227 * 1024;
 }
 
 cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
@@ -525,9 +592,14 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
                              (uint32_t)(8 * T), CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess)
         return e;
-    const Smem L = T == 1 ? smem_layout<8>(p.KS, p.rp, p.R1p)
-                          : (T == 2 ? smem_layout<16>(p.KS, p.rp, p.R1p) : smem_layout<32>(p.KS, p.rp, p.R1p));
-    const size_t smem = L.total + 1024;
+    // push the partial tiles when the receive slots fit, else pull them over DSMEM
+    auto layout = [&](int nslots) {
+        return T == 1 ? smem_layout<8>(p.KS, p.rp, p.R1p, nslots)
+                      : (T == 2 ? smem_layout<16>(p.KS, p.rp, p.R1p, nslots)
+                                : smem_layout<32>(p.KS, p.rp, p.R1p, nslots));
+    };
+    p.push = layout(CS - 1).total + 1024 <= 227 * 1024 ? 1 : 0;
+    const size_t smem = layout(p.push ? CS - 1 : 0).total + 1024;
     const void *fn = T == 1 ? kernel_ptr<1>() : (T == 2 ? kernel_ptr<2>() : kernel_ptr<4>());
     e = raise_smem_limit(fn, smem);
     if (e != cudaSuccess)
