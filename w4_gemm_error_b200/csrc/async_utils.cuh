@@ -241,6 +241,13 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr)
     return v;
 }
 
+// Counter increment that releases (cumulatively) every write this thread has
+// observed, including its CTA's writes ordered before it by a CTA barrier.
+__device__ __forceinline__ void red_release_gpu_add(unsigned *p, unsigned v)
+{
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *p)
 {
     unsigned v;

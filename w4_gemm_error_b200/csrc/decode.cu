@@ -19,9 +19,10 @@
 //  * weight rows sit on the 16-row side of mma.sync m16n8k16 and tokens on
 //    the 8-column side, so a code is read once for up to 32 tokens; the
 //    codes are dequantised in registers to exact (q - z) bf16 pairs (two
-//    nibbles 16 bits apart per register), and the activations are paired to
-//    match with one byte permute per register, the k order inside the MMA
-//    being permuted accordingly;
+//    nibbles 16 bits apart per register, set into the mantissa of 128.0 and
+//    offset by one bf16 fma), and the activations are paired to match with
+//    one byte permute per register, the k order inside the MMA being
+//    permuted accordingly;
 //  * the K split is summed inside the cluster, in rank order
 //    (deterministic), with no global round trip: the other CTAs push their
 //    partial tiles into receive slots of the first CTA (st.async, counted on
@@ -30,10 +31,11 @@
 //    CTA pulls the tiles over distributed shared memory between two cluster
 //    barriers instead;
 //  * the EC down-projection u = x . [w_g, A] runs on R1p/16 extra clusters
-//    of the same grid (the first ones) with the same slicing; they publish u
-//    in global memory behind a counter, and the 64-row clusters read it for
-//    their epilogue
-//        y[t,n] = bf16( s[n] * acc[t,n] + sum_j g_t u[t,j] B[j,n] ),
+//    of the same grid (the first ones) with the same slicing; each of their
+//    CTAs publishes its partial of u in global memory and counts it with a
+//    release increment, and the first CTA of each 64-row cluster, once the
+//    count is complete, sums the partials in rank order for its epilogue
+//        y[t,n] = bf16( s[n] * acc[t,n] + g_t * sum_j u[t,1+j] B[j,n] ),
 //        g_t = 1 / (1 + exp(-(u[t,0] + b_g))),
 //    with a bounded wait (about a second) that records a timeout in the
 //    handle's status word instead of hanging.
@@ -63,8 +65,8 @@ struct DecodeParams {
     const float *s;
     const uint8_t *z;
     uint16_t *y;
-    float *ws_u;          // [R1p][kUStride] fp32
-    unsigned *flags;      // [0] u clusters published, [1] row clusters done with u
+    float *ws_u;          // [CS][R1p][kUStride] fp32: one partial of u per rank
+    unsigned *flags;      // [0] EC CTAs published, [1] row clusters done with u
     int *status;
     int64_t M, N, Kp;
     int KS, nch;          // k per CTA (a multiple of 256), code chunks per CTA
@@ -88,8 +90,8 @@ __host__ __device__ inline Smem smem_layout(int KS, int rp, int R1p, int nslots)
     m.x = m.codes + 32 * KS;                       // 2*TOK*KS bytes: activation sub-tiles
     m.bt = m.x + 2 * TOK * KS;                     // 128*rp bytes: B^T rows of the cluster
     m.red = m.bt + 128 * rp;                       // 512*TOK bytes: partial tiles
-    m.u = m.red + 512 * TOK;                       // u [R1p][TOK], g [TOK], v [TOK][rp] (fp32)
-    m.recv = (m.u + 4 * R1p * TOK + 4 * TOK * (rp + 1) + 15) & ~15u;
+    m.u = m.red + 512 * TOK;                       // u0 [TOK], uT [TOK][rp] (fp32)
+    m.recv = (m.u + 4 * TOK * (rp + 1) + 15) & ~15u;
     m.total = m.recv + nslots * 256 * TOK;
     return m;
 }
@@ -99,41 +101,19 @@ __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) { re
 constexpr int kThreads = 256;   // 8 warps: two per 16-row group, splitting the sub-blocks
 constexpr int kEcWarp = kThreads / 32 - 1;
 
-// One warp: wait (bounded) until the EC clusters have published u, copy u
-// [R1p][TOK] into shared memory, then g [TOK] and v [TOK][rp] = g * u[1..r].
-template <int TOK>
-__device__ __forceinline__ void fetch_u(const DecodeParams &p, float *us, float *gs, float *vv, int lane)
+// Bounded wait (one thread) until every CTA of the EC clusters has published
+// its partial u; false if it ran out (the timeout is recorded in the status).
+__device__ __forceinline__ bool wait_u_published(const DecodeParams &p, unsigned expected)
 {
-    int good = 1;
-    if (lane == 0) {
-        const long long t0 = clock64();
-        while (ld_acquire_gpu(&p.flags[0]) < (unsigned)p.JB) {
-            if (clock64() - t0 > kWaitBudgetCycles) {
-                atomicOr(p.status, kStatusTimeout);
-                good = 0;
-                break;
-            }
-            __nanosleep(32);
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(&p.flags[0]) < expected) {
+        if (clock64() - t0 > kWaitBudgetCycles) {
+            atomicOr(p.status, kStatusTimeout);
+            return false;
         }
+        __nanosleep(32);
     }
-    good = __shfl_sync(0xffffffffu, good, 0);
-    for (int e = lane; e < p.R1p * TOK; e += 32) {
-        const int row = e / TOK, t = e - row * TOK;
-        us[e] = good ? __ldcg(p.ws_u + row * kUStride + t) : 0.f;
-    }
-    __syncwarp();
-    if (lane == 0 && atomicAdd(&p.flags[1], 1u) == (unsigned)(p.NC - 1)) {
-        // every 64-row cluster has read u: reset for the next forward
-        p.flags[1] = 0u;
-        p.flags[0] = 0u;
-    }
-    for (int t = lane; t < TOK; t += 32)
-        gs[t] = 1.0f / (1.0f + expf(-(us[t] + p.b_g)));
-    __syncwarp();
-    for (int e = lane; e < TOK * p.rp; e += 32) {
-        const int t = e / p.rp, j = e - t * p.rp;
-        vv[e] = j < p.r ? gs[t] * us[(1 + j) * TOK + t] : 0.f;
-    }
+    return true;
 }
 
 template <int T>
@@ -165,7 +145,6 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     const uint32_t bar_bt = smem_addr(&bars[kMaxChunks + 1]);
     const uint32_t bar_recv = smem_addr(&bars[kMaxChunks + 2]);
     const int n0 = is_u ? 0 : (cluster - p.JB) * kRows;
-    const int tile_rows = is_u ? 16 : kRows;
 
     // loads that do not depend on earlier kernels are issued before waiting
     // for them: the epilogue scale of this thread's row and the zero points
@@ -178,8 +157,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         for (int c = 0; c < kMaxChunks + 3; ++c)
             mbar_init(bar_chunk + 8 * c, 1);
         fence_mbarrier_init_cluster();
-        if (push && rank == 0 && CS > 1)
-            mbar_expect_tx(bar_recv, (uint32_t)((CS - 1) * tile_rows * TOK * 4));
+        if (push && !is_u && rank == 0 && CS > 1)
+            mbar_expect_tx(bar_recv, (uint32_t)((CS - 1) * kRows * TOK * 4));
         // the weights do not depend on earlier kernels: start them now
         for (int c = 0; c < nch; ++c) {
             const uint32_t bar = bar_chunk + 8 * c;
@@ -201,15 +180,20 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     __syncthreads();
     if (push)
         cluster_arrive_relaxed();   // the receive barrier of the first CTA is initialised
+    __shared__ int s_xok;
     if (tid == 0) {
         // the activations are written by the previous kernel in the stream
         pdl_wait();
         mbar_expect_tx(bar_x, 2 * TOK * kChunk * nch);
         for (int i = 0; i < nsub; ++i)
             tma_load_2d(base + L.x + i * (TOK * 128), &tm_x, k0 + 64 * i, 0, bar_x);
+        s_xok = wait_bounded(bar_x, 0) ? 1 : 0;
     }
-
-    bool ok = wait_bounded(bar_x, 0);
+    // the other threads sleep in this barrier instead of polling (they would
+    // take issue slots from the previous layer's CTAs on the same SM); their
+    // own wait below then returns at once and orders their reads after the copy
+    __syncthreads();
+    bool ok = s_xok != 0 && wait_bounded(bar_x, 0);
 
     // two accumulator sets (even / odd code word) halve the MMA dependency chains
     float acc[T][4], acc2[T][4];
@@ -226,8 +210,13 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         const uint32_t nbg = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + zg_raw)));
         const uint32_t nbh = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + zh_raw)));
         const uint32_t negg = nbg | (nbg << 16), negh = nbh | (nbh << 16);
-        for (int c = 0; c < nch && ok; ++c) {
-            ok = wait_bounded(bar_chunk + 8 * c, 0);
+        // the codes were requested before the wait for the previous kernel and
+        // have normally landed: one wait for all, so that no compiler barrier
+        // sits inside the loop
+        for (int c = 0; c < nch; ++c)
+            ok = ok && wait_bounded(bar_chunk + 8 * c, 0);
+#pragma unroll 2
+        for (int c = 0; c < (ok ? nch : 0); ++c) {
             const uint8_t *ctile = bp + L.codes + c * 8192;
 #pragma unroll
             for (int sb2 = 0; sb2 < 2; ++sb2) {
@@ -255,9 +244,11 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 #pragma unroll
                     for (int n = 0; n < T; ++n) {
                         const uint4 v = xv[n][j];
+                        const uint32_t b0 = prmt(v.x, v.z, 0x5410), b1 = prmt(v.x, v.z, 0x7632);
+                        const uint32_t b2 = prmt(v.y, v.w, 0x5410), b3 = prmt(v.y, v.w, 0x7632);
                         float (&a)[4] = j ? acc2[n] : acc[n];
-                        mma_bf16_16816(a, g0, h0, g1, h1, prmt(v.x, v.z, 0x5410), prmt(v.x, v.z, 0x7632));
-                        mma_bf16_16816(a, g2, h2, g3, h3, prmt(v.y, v.w, 0x5410), prmt(v.y, v.w, 0x7632));
+                        mma_bf16_16816(a, g0, h0, g1, h1, b0, b1);
+                        mma_bf16_16816(a, g2, h2, g3, h3, b2, b3);
                     }
                 }
             }
@@ -277,8 +268,11 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             mine[(rg + 8) * TOK + col + 1] = acc[n][3];
         }
         __syncthreads();
-        for (int e = tid; e < kRows * TOK; e += kThreads)
+#pragma unroll
+        for (int i = 0; i < TOK / 4; ++i) {
+            const int e = tid + kThreads * i;   // row e / TOK, token e % TOK
             red[e] = red[e] + red[kRows * TOK + e];
+        }
     } else {
         // ---- 16 rows of G = [w_g; A^T]: warp w takes the 64-wide sub-tiles i = w (mod 8)
         for (int i = warp; i < nsub && ok; i += 8) {
@@ -341,19 +335,33 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             wait_bounded(bar_bt, 0);
     }
 
+    if (is_u) {
+        // ---- publish this CTA's partial of u rows 16*cluster .. +15 (all TOK
+        // columns); the 64-row clusters sum the CS partials in rank order
+        float *dst = p.ws_u + ((int64_t)rank * p.R1p + 16 * cluster) * kUStride;
+        for (int e = tid; e < 16 * TOK; e += kThreads) {
+            const int row = e / TOK, t = e - row * TOK;
+            dst[row * kUStride + t] = red[e];
+        }
+        __syncthreads();
+        if (tid == 0)
+            red_release_gpu_add(&p.flags[0], 1u);
+        if (push)
+            cluster_wait();   // pairs with the arrive after the barrier set-up
+        return;
+    }
+
     // ---- sum the K split over the cluster, in rank order, in the first CTA.
-    // In the first CTA of a 64-row cluster with an EC, the last warp fetches u
-    // meanwhile.
-    float *us = reinterpret_cast<float *>(bp + L.u);   // u [R1p][TOK]
-    float *gs = us + p.R1p * TOK;                      // g [TOK]
-    float *vv = gs + TOK;                              // v [TOK][rp] = g * u
-    const bool ec_warp = !is_u && rank == 0 && p.JB > 0 && warp == kEcWarp;
-    const int nsum = (!is_u && p.JB > 0) ? kThreads - 32 : kThreads;
-    const int tile4 = tile_rows * TOK / 4;
+    // With an EC, the last warp of the first CTA meanwhile waits until u is
+    // published.
+    const bool ec_warp = rank == 0 && p.JB > 0 && warp == kEcWarp;
+    const int nsum = p.JB > 0 ? kThreads - 32 : kThreads;
+    constexpr int tile4 = kRows * TOK / 4;
+    __shared__ int s_good;
     if (push) {
         cluster_wait();   // every receive barrier of the cluster is initialised
         if (rank != 0) {
-            const uint32_t dst = map_to_rank(base + L.recv + (rank - 1) * (tile_rows * TOK * 4), 0);
+            const uint32_t dst = map_to_rank(base + L.recv + (rank - 1) * (kRows * TOK * 4), 0);
             const uint32_t rbar = map_to_rank(bar_recv, 0);
             for (int e4 = tid; e4 < tile4; e4 += kThreads)
                 st_async_f4(dst + 16 * e4, reinterpret_cast<const float4 *>(red)[e4], rbar);
@@ -362,10 +370,10 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             return;
         }
         if (ec_warp) {
-            fetch_u<TOK>(p, us, gs, vv, lane);
-        } else if (CS > 1) {
-            if (!wait_bounded(bar_recv, 0) && tid == 0)
-                atomicOr(p.status, kStatusTimeout);
+            if (lane == 0)
+                s_good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
+        } else if (CS > 1 && !wait_bounded(bar_recv, 0) && tid == 0) {
+            atomicOr(p.status, kStatusTimeout);
         }
         cluster_arrive();     // the tiles have landed: the other CTAs may leave
         const float4 *slots = reinterpret_cast<const float4 *>(bp + L.recv);
@@ -384,29 +392,28 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     } else {
         __syncthreads();
         cluster_sync();
-        if (rank == 0) {
-            if (ec_warp) {
-                fetch_u<TOK>(p, us, gs, vv, lane);
-            } else {
-                const uint32_t red_addr = base + L.red;
-                for (int e4 = tid; e4 < tile4; e4 += nsum) {
-                    // issue every remote load before summing (in rank order)
-                    float4 o[8];
+        if (ec_warp) {
+            if (lane == 0)
+                s_good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
+        } else if (rank == 0) {
+            const uint32_t red_addr = base + L.red;
+            for (int e4 = tid; e4 < tile4; e4 += nsum) {
+                // issue every remote load before summing (in rank order)
+                float4 o[8];
 #pragma unroll
-                    for (int q = 1; q < 8; ++q)
-                        if (q < CS)
-                            o[q] = ld_dsmem_f4(map_to_rank(red_addr + 16 * e4, (uint32_t)q));
-                    float4 s = reinterpret_cast<const float4 *>(red)[e4];
+                for (int q = 1; q < 8; ++q)
+                    if (q < CS)
+                        o[q] = ld_dsmem_f4(map_to_rank(red_addr + 16 * e4, (uint32_t)q));
+                float4 s = reinterpret_cast<const float4 *>(red)[e4];
 #pragma unroll
-                    for (int q = 1; q < 8; ++q)
-                        if (q < CS) {
-                            s.x += o[q].x;
-                            s.y += o[q].y;
-                            s.z += o[q].z;
-                            s.w += o[q].w;
-                        }
-                    reinterpret_cast<float4 *>(red)[e4] = s;
-                }
+                for (int q = 1; q < 8; ++q)
+                    if (q < CS) {
+                        s.x += o[q].x;
+                        s.y += o[q].y;
+                        s.z += o[q].z;
+                        s.w += o[q].w;
+                    }
+                reinterpret_cast<float4 *>(red)[e4] = s;
             }
         }
         cluster_sync();  // the other CTAs' shared memory is no longer read
@@ -415,19 +422,38 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     }
     __syncthreads();
 
-    if (is_u) {
-        // publish u rows 16*cluster .. +15 for all TOK token columns
-        for (int e = tid; e < 16 * TOK; e += kThreads) {
+    // ---- EC: u = sum over the CS published partials (rank order), as u0 [TOK]
+    // (gate logits) and uT [TOK][rp] (u[1 + j][t] transposed, zero for j >= r)
+    float *u0 = reinterpret_cast<float *>(bp + L.u);
+    float *uT = u0 + TOK;
+    if (p.JB > 0) {
+        const bool good = s_good != 0;
+        for (int e = tid; e < (1 + p.r) * TOK; e += kThreads) {
             const int row = e / TOK, t = e - row * TOK;
-            p.ws_u[(16 * cluster + row) * kUStride + t] = red[e];
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                v[q] = (q < CS && good) ? __ldcg(p.ws_u + ((int64_t)q * p.R1p + row) * kUStride + t) : 0.f;
+            float u = v[0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q)
+                if (q < CS)
+                    u += v[q];
+            if (row == 0)
+                u0[t] = u;
+            else
+                uT[t * p.rp + row - 1] = u;
         }
-        __threadfence();
+        for (int e = tid; e < TOK * (p.rp - p.r); e += kThreads) {
+            const int t = e / (p.rp - p.r), j = p.r + e - t * (p.rp - p.r);
+            uT[t * p.rp + j] = 0.f;
+        }
         __syncthreads();
-        if (tid == 0)
-            atomicAdd(&p.flags[0], 1u);
-        if (push)
-            cluster_wait();
-        return;
+        if (tid == 0 && atomicAdd(&p.flags[1], 1u) == (unsigned)(p.NC - 1)) {
+            // every 64-row cluster has read u: reset for the next forward
+            p.flags[1] = 0u;
+            p.flags[0] = 0u;
+        }
     }
 
     // ---- epilogue of a 64-row cluster
@@ -440,8 +466,12 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     for (int i = 0; i < TOK / 4; ++i)
         out[i] = s_epi * red[row * TOK + th + 4 * i];
     if (p.JB > 0) {
-        // corr = sum_j v[t][j] * B^T[n][j]: the B^T row in 16-byte pieces from shared memory,
-        // v broadcast from shared memory
+        // corr = g_t * sum_j u[1 + j][t] * B^T[n][j]: the B^T row in 16-byte pieces,
+        // u broadcast, both from shared memory
+        float corr[TOK / 4];
+#pragma unroll
+        for (int i = 0; i < TOK / 4; ++i)
+            corr[i] = 0.f;
         const uint16_t *btrow = reinterpret_cast<const uint16_t *>(bp + L.bt) + row * p.rp;
         for (int j0 = 0; j0 < p.rp; j0 += 8) {
             const uint4 bv = *reinterpret_cast<const uint4 *>(btrow + j0);
@@ -449,11 +479,16 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                                  bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
 #pragma unroll
             for (int i = 0; i < TOK / 4; ++i) {
-                const float4 *vt = reinterpret_cast<const float4 *>(vv + (th + 4 * i) * p.rp + j0);
-                const float4 v0 = vt[0], v1 = vt[1];
-                out[i] += v0.x * bj[0] + v0.y * bj[1] + v0.z * bj[2] + v0.w * bj[3] + v1.x * bj[4] +
-                          v1.y * bj[5] + v1.z * bj[6] + v1.w * bj[7];
+                const float4 *ut = reinterpret_cast<const float4 *>(uT + (th + 4 * i) * p.rp + j0);
+                const float4 v0 = ut[0], v1 = ut[1];
+                corr[i] += v0.x * bj[0] + v0.y * bj[1] + v0.z * bj[2] + v0.w * bj[3] + v1.x * bj[4] +
+                           v1.y * bj[5] + v1.z * bj[6] + v1.w * bj[7];
             }
+        }
+#pragma unroll
+        for (int i = 0; i < TOK / 4; ++i) {
+            const float g = 1.0f / (1.0f + expf(-(u0[th + 4 * i] + p.b_g)));
+            out[i] += g * corr[i];
         }
     }
 #pragma unroll
@@ -552,7 +587,8 @@ void decode_free(DecodeWork &w)
     w.maps = nullptr;
 }
 
-size_t decode_u_floats(const Packed &pk) { return (size_t)pk.R1p * kUStride; }
+// one partial of u per rank of an EC cluster (at most 8 ranks)
+size_t decode_u_floats(const Packed &pk) { return (size_t)8 * pk.R1p * kUStride; }
 
 cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, bool ec, const DecodeWork &w,
                           int *status, cudaStream_t st, int num_sms)

@@ -65,7 +65,7 @@ int prepass_counters(int64_t max_M);
 // and EC up-projection in the epilogue (when `ec` is set).
 struct DecodeWork {
     void *maps;           // tensor maps of the packed operands (host memory)
-    float *ws_u;          // [R1p][32] published EC down-projection
+    float *ws_u;          // [8][R1p][32] published partials of the EC down-projection
     unsigned *flags;      // two counters, zero between calls
 };
 constexpr int kDecodeMaxTokens = 32;   // tokens per launch
