@@ -75,6 +75,39 @@ def packed_bytes(K, N, r):
     return N * K // 2 + 5 * N + 2 * K * (r + 1) + 2 * r * N
 
 
+# DRAM bytes (read + write) per launch of each workload's dominant kernel, by
+# batch size, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum)
+# of the kernel sources whose SHA-256 prefix is given; the summaries under
+# profiles/ give the commands.  Reported only while those sources are unchanged.
+TRAFFIC = {
+    "decode_qo_4096x4096_r32": dict(
+        kernel="decode_w4ec_kernel",
+        files=("decode.cu", "async_utils.cuh", "device_utils.cuh", "kernels.h"), sha="6106bb890d1d1383",
+        bytes={1: 9.129e6, 4: 9.1515e6, 16: 9.253e6},
+        profile="profiles/decode_w4ec_kernel_decode_qo_4096x4096_r32.md"),
+    "prefill_mlp_4096x14336_r64": dict(
+        kernel="tc_w4ec_kernel",
+        files=("tc_gemm.cu", "tc_gemm.h", "async_utils.cuh", "device_utils.cuh"), sha="6cc58f664e8fa866",
+        bytes={2048: 70.118e6, 4096: 156.885e6},
+        profile="profiles/tc_w4ec_kernel_prefill_mlp_4096x14336_r64.md"),
+}
+
+
+def traffic_per_launch(workload, Ms):
+    """Mean measured DRAM bytes per launch over the step's batch sizes, or None."""
+    import hashlib
+    t = TRAFFIC.get(workload)
+    if t is None or any(M not in t["bytes"] for M in Ms):
+        return None
+    h = hashlib.sha256()
+    for f in t["files"]:
+        with open(os.path.join(ROOT, "w4_gemm_error_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    if h.hexdigest()[:16] != t["sha"]:
+        return None
+    return round(sum(t["bytes"][M] for M in Ms) / len(Ms))
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -279,13 +312,16 @@ def run_ours(args, rank, world, local_rank):
     peaks = load_peaks()
     if wl["kind"] == "decode":
         roof = {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": round(per_gpu / peaks["hbm"], 4), "traffic": None,
+                "frac": round(per_gpu / peaks["hbm"], 4), "traffic": traffic_per_launch(args.workload, Ms),
+                "alg_bytes_per_launch": round(sum(alg_bytes(M, K, N, r) for M in Ms) / len(Ms)),
                 "kernel": "decode_w4ec_kernel (one launch per forward): per-forward time in the chained stack",
                 "peak_source": peaks["source"]}
     else:
         pk = peaks["bf16_sustained"]
         roof = {"bound": "tensor", "achieved": round(per_gpu, 1), "peak": pk, "unit": "TFLOP/s",
-                "frac": round(per_gpu / pk, 4), "traffic": None, "kernel": "tc path: per-forward time",
+                "frac": round(per_gpu / pk, 4), "traffic": traffic_per_launch(args.workload, Ms),
+                "kernel": "tc_w4ec_kernel: per-forward time, which also holds the tc_prepass_kernel launch "
+                          "(about 5% of the launch list), so the kernel's own rate is higher",
                 "peak_source": peaks["source"] + " (sustained)"}
 
     launches_per_forward = {}
