@@ -5,24 +5,28 @@
 // into the low-bit GEMM.  For a few tokens the layer is bound by reading the
 // int4 codes from HBM, and in a decode pass its critical path is the chain
 // "previous layer done -> this layer done", so the kernel is built to stream
-// the weights before that chain starts and to keep the chain short:
+// the weights from the start and to keep that chain short:
 //
 //  * one kernel per forward; a cluster of CS CTAs owns 64 weight rows, each
-//    CTA one K/CS slice of them;
-//  * before waiting for the previous kernel (programmatic dependent launch)
-//    every CTA starts TMA copies of its whole slice of codes (and the
-//    cluster's first CTA those of the B^T rows of its epilogue), so the
-//    weight stream overlaps the previous layer; only the activations are
-//    fetched after the wait;
-//  * eight warps per CTA, two per 16-row group splitting the 64-wide
-//    sub-blocks, so the dequantise-MMA chains of one warp hide another's;
+//    CTA one K/CS slice of them, sized so that the grid is one wave of about
+//    two CTAs per SM;
+//  * a producer warp streams the slice through a ring of shared-memory
+//    stages (one 8 KB block of codes and the matching activations per
+//    256 k), with full and empty mbarriers; before waiting for the previous
+//    kernel (programmatic dependent launch) it fills every stage's codes (a
+//    short slice is then entirely resident), and the consumers sleep in a CTA
+//    barrier until the activations are on their way;
+//  * eight consumer warps, two per 16-row group splitting the 64-wide
+//    sub-blocks of each stage, so the dequantise-MMA chains of one warp hide
+//    another's;
 //  * weight rows sit on the 16-row side of mma.sync m16n8k16 and tokens on
 //    the 8-column side, so a code is read once for up to 32 tokens; the
 //    codes are dequantised in registers to exact (q - z) bf16 pairs (two
 //    nibbles 16 bits apart per register, set into the mantissa of 128.0 and
-//    offset by one bf16 fma), and the activations are paired to match with
-//    one byte permute per register, the k order inside the MMA being
-//    permuted accordingly;
+//    offset by one bf16 fma); the stored nibble order makes each pair two
+//    consecutive k, so the activations enter the MMA as they lie in shared
+//    memory (each thread takes 16 consecutive k of its rows, the k order
+//    inside the MMA being permuted accordingly);
 //  * the K split is summed inside the cluster, in rank order
 //    (deterministic), with no global round trip: the other CTAs push their
 //    partial tiles into receive slots of the first CTA (st.async, counted on
@@ -49,10 +53,16 @@
 namespace spear {
 namespace {
 
-constexpr int kRows = 64;       // weight rows per cluster (four warps x 16)
-constexpr int kChunk = 256;     // k per code chunk (one 8 KB TMA box of 64 rows)
-constexpr int kMaxChunks = 8;   // so K/CS <= 2048
-constexpr int kUStride = 32;    // token stride of the published u rows
+constexpr int kRows = 64;         // weight rows per cluster (four warps x 16)
+constexpr int kChunk = 256;       // k per stage (one 8 KB TMA box of 64 rows of codes)
+constexpr int kMaxStages = 8;     // ring depth limit
+constexpr int kUStride = 32;      // token stride of the published u rows
+constexpr int kConsumers = 256;   // 8 consumer warps: two per 16-row group
+constexpr int kThreads = kConsumers + 32;   // + one producer warp
+constexpr int kProducerWarp = kConsumers / 32;
+constexpr int kEcWarp = kProducerWarp - 1;  // consumer warp that waits for u
+// shared memory per CTA that keeps two CTAs per SM resident
+constexpr int kSmemPerCta = 110 * 1024;
 
 struct Maps {
     CUtensorMap codes;    // tiled codes, one box = one 8 KB block (64 rows x 256 k), 128B swizzle
@@ -69,26 +79,35 @@ struct DecodeParams {
     unsigned *flags;      // [0] EC CTAs published, [1] row clusters done with u
     int *status;
     int64_t M, N, Kp;
-    int KS, nch;          // k per CTA (a multiple of 256), code chunks per CTA
+    int KS, nch;          // k per CTA (a multiple of 256), chunks of 256 k per CTA
+    int S;                // ring stages
     int JB, NC;           // EC clusters, 64-row clusters
     int r, rp, R1p;
     int push;             // partial tiles pushed into receive slots of the first CTA
     float b_g;
 };
 
+// Bytes of one ring stage: the codes of 64 rows x 256 k (or 16 G rows x
+// 256 k as four 2 KB boxes), then the activations as four 64-k sub-tiles of
+// TOK rows x 128 bytes.
+template <int TOK>
+__host__ __device__ constexpr uint32_t stage_bytes()
+{
+    return 8192 + 4 * TOK * 128;
+}
+
 struct Smem {
-    uint32_t codes, x, bt, red, u, recv;   // byte offsets from the 1024-aligned base
+    uint32_t ring, bt, red, u, recv;   // byte offsets from the 1024-aligned base
     uint32_t total;
 };
 
-// nslots receive slots of one partial tile (64 rows x TOK fp32) each.
+// S ring stages; nslots receive slots of one partial tile (64 rows x TOK fp32) each.
 template <int TOK>
-__host__ __device__ inline Smem smem_layout(int KS, int rp, int R1p, int nslots)
+__host__ __device__ inline Smem smem_layout(int S, int rp, int nslots)
 {
     Smem m;
-    m.codes = 0;                                   // 32*KS bytes: codes (64 rows) or G (16 rows bf16)
-    m.x = m.codes + 32 * KS;                       // 2*TOK*KS bytes: activation sub-tiles
-    m.bt = m.x + 2 * TOK * KS;                     // 128*rp bytes: B^T rows of the cluster
+    m.ring = 0;
+    m.bt = m.ring + S * stage_bytes<TOK>();        // 128*rp bytes: B^T rows of the cluster
     m.red = m.bt + 128 * rp;                       // 512*TOK bytes: partial tiles
     m.u = m.red + 512 * TOK;                       // u0 [TOK], uT [TOK][rp] (fp32)
     m.recv = (m.u + 4 * TOK * (rp + 1) + 15) & ~15u;
@@ -97,9 +116,6 @@ __host__ __device__ inline Smem smem_layout(int KS, int rp, int R1p, int nslots)
 }
 
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity) { return mbar_wait_bounded(bar, parity); }
-
-constexpr int kThreads = 256;   // 8 warps: two per 16-row group, splitting the sub-blocks
-constexpr int kEcWarp = kThreads / 32 - 1;
 
 // Bounded wait (one thread) until every CTA of the EC clusters has published
 // its partial u; false if it ran out (the timeout is recorded in the status).
@@ -116,62 +132,86 @@ __device__ __forceinline__ bool wait_u_published(const DecodeParams &p, unsigned
     return true;
 }
 
+// Register budget: three CTAs per SM up to 16 tokens (the grid is about two
+// per SM, and the next layer's kernel starts beside it), two at 32 tokens.
 template <int T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, T == 4 ? 2 : 3)
 decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_g,
                    const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_x,
                    DecodeParams p, int CS)
 {
     constexpr int TOK = 8 * T;
+    constexpr uint32_t kStage = stage_bytes<TOK>();
+    constexpr uint32_t kXBytes = 4 * TOK * 128;
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[kMaxChunks + 3];
+    // per stage: codes landed, activations landed, stage free; then B^T, K-split receive
+    __shared__ __align__(8) uint64_t bars[3 * kMaxStages + 2];
+    __shared__ int s_good;
 
     pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, cl = lane & 3;
+    const bool producer = warp == kProducerWarp;
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const bp = smem_raw + (base - raw);
     const bool push = p.push != 0;
-    const Smem L = smem_layout<TOK>(p.KS, p.rp, p.R1p, push ? CS - 1 : 0);
+    const Smem L = smem_layout<TOK>(p.S, p.rp, push ? CS - 1 : 0);
     const uint32_t rank = cluster_ctarank();
     const int cluster = blockIdx.x / CS;
     const bool is_u = cluster < p.JB;
     const int k0 = (int)rank * p.KS;
     // the last ranks may hold a shorter (or empty) slice when K/256 is not a multiple of CS
     const int nch = max(0, min(p.nch, (int)((p.Kp - k0) / kChunk)));
-    const int nsub = 4 * nch;
-    const uint32_t bar_chunk = smem_addr(&bars[0]);
-    const uint32_t bar_x = smem_addr(&bars[kMaxChunks]);
-    const uint32_t bar_bt = smem_addr(&bars[kMaxChunks + 1]);
-    const uint32_t bar_recv = smem_addr(&bars[kMaxChunks + 2]);
+    const int S = p.S;
+    const int first = min(S, nch);   // chunks whose stages are filled before the dependency wait
+    const uint32_t bar_full_w = smem_addr(&bars[0]);
+    const uint32_t bar_full_x = smem_addr(&bars[kMaxStages]);
+    const uint32_t bar_empty = smem_addr(&bars[2 * kMaxStages]);
+    const uint32_t bar_bt = smem_addr(&bars[3 * kMaxStages]);
+    const uint32_t bar_recv = smem_addr(&bars[3 * kMaxStages + 1]);
     const int n0 = is_u ? 0 : (cluster - p.JB) * kRows;
 
-    // loads that do not depend on earlier kernels are issued before waiting
-    // for them: the epilogue scale of this thread's row and the zero points
-    // of its two MMA rows
-    const float s_epi = (!is_u && rank == 0) ? __ldg(p.s + n0 + (tid & (kRows - 1))) : 0.f;
+    // loads that do not depend on earlier kernels are issued first: the
+    // epilogue scale of this thread's row and the zero points of its MMA rows
+    const float s_epi = (!is_u && rank == 0 && !producer) ? __ldg(p.s + n0 + (tid & (kRows - 1))) : 0.f;
     const int rg = 16 * (warp & 3) + gid;  // MMA rows rg and rg + 8 (64-row clusters)
-    const uint32_t zg_raw = is_u ? 0u : (uint32_t)__ldg(p.z + n0 + rg);
-    const uint32_t zh_raw = is_u ? 0u : (uint32_t)__ldg(p.z + n0 + rg + 8);
-    if (tid == 0) {
-        for (int c = 0; c < kMaxChunks + 3; ++c)
-            mbar_init(bar_chunk + 8 * c, 1);
+    const uint32_t zg_raw = (is_u || producer) ? 0u : (uint32_t)__ldg(p.z + n0 + rg);
+    const uint32_t zh_raw = (is_u || producer) ? 0u : (uint32_t)__ldg(p.z + n0 + rg + 8);
+
+    // producer: chunk c of this CTA's slice goes to stage st = c % S
+    auto issue_codes = [&](int c, int st) {
+        const uint32_t dst = base + L.ring + st * kStage;
+        const uint32_t bar = bar_full_w + 8 * st;
+        mbar_expect_tx(bar, 8192);
+        if (is_u) {
+            for (int i = 0; i < 4; ++i)
+                tma_load_2d(dst + i * 2048, &tm_g, k0 + c * kChunk + i * 64, 16 * cluster, bar);
+        } else {
+            tma_load_3d(dst, &tm_codes, 0, 0, (n0 / kRows) * (int)(p.Kp / kChunk) + (k0 / kChunk) + c, bar);
+        }
+    };
+    auto issue_x = [&](int c, int st) {
+        const uint32_t dst = base + L.ring + st * kStage + 8192;
+        const uint32_t bar = bar_full_x + 8 * st;
+        mbar_expect_tx(bar, kXBytes);
+        for (int i = 0; i < 4; ++i)
+            tma_load_2d(dst + i * (TOK * 128), &tm_x, k0 + c * kChunk + 64 * i, 0, bar);
+    };
+
+    if (producer && lane == 0) {
+        for (int i = 0; i < kMaxStages; ++i) {
+            mbar_init(bar_full_w + 8 * i, 1);
+            mbar_init(bar_full_x + 8 * i, 1);
+            mbar_init(bar_empty + 8 * i, kConsumers / 32);
+        }
+        mbar_init(bar_bt, 1);
+        mbar_init(bar_recv, 1);
         fence_mbarrier_init_cluster();
         if (push && !is_u && rank == 0 && CS > 1)
             mbar_expect_tx(bar_recv, (uint32_t)((CS - 1) * kRows * TOK * 4));
-        // the weights do not depend on earlier kernels: start them now
-        for (int c = 0; c < nch; ++c) {
-            const uint32_t bar = bar_chunk + 8 * c;
-            mbar_expect_tx(bar, 8192);
-            if (is_u) {
-                for (int i = 0; i < 4; ++i)
-                    tma_load_2d(base + L.codes + c * 8192 + i * 2048, &tm_g, k0 + c * kChunk + i * 64, 16 * cluster,
-                                bar);
-            } else {
-                tma_load_3d(base + L.codes + c * 8192, &tm_codes, 0, 0,
-                            (n0 / kRows) * (int)(p.Kp / kChunk) + (k0 / kChunk) + c, bar);
-            }
-        }
+        // the weights do not depend on earlier kernels: fill every stage now
+        for (int c = 0; c < first; ++c)
+            issue_codes(c, c);
         if (!is_u && rank == 0 && p.rp > 0) {
             mbar_expect_tx(bar_bt, 128 * p.rp);   // B^T rows of the cluster, for the epilogue
             tma_load_2d(base + L.bt, &tm_bt, 0, n0, bar_bt);
@@ -180,21 +220,20 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     __syncthreads();
     if (push)
         cluster_arrive_relaxed();   // the receive barrier of the first CTA is initialised
-    __shared__ int s_xok;
-    if (tid == 0) {
+    int issued = 0;                 // producer: chunks whose codes and activations are requested
+    if (producer && lane == 0) {
         // the activations are written by the previous kernel in the stream
         pdl_wait();
-        mbar_expect_tx(bar_x, 2 * TOK * kChunk * nch);
-        for (int i = 0; i < nsub; ++i)
-            tma_load_2d(base + L.x + i * (TOK * 128), &tm_x, k0 + 64 * i, 0, bar_x);
-        s_xok = wait_bounded(bar_x, 0) ? 1 : 0;
+        for (int c = 0; c < first; ++c)
+            issue_x(c, c);
+        issued = first;
     }
-    // the other threads sleep in this barrier instead of polling (they would
-    // take issue slots from the previous layer's CTAs on the same SM); their
-    // own wait below then returns at once and orders their reads after the copy
+    // the consumers sleep in this barrier, rather than poll, while the
+    // producer waits for the previous kernel (polling would take issue slots
+    // from the previous layer's CTAs on the same SM)
     __syncthreads();
-    bool ok = s_xok != 0 && wait_bounded(bar_x, 0);
 
+    bool ok = true;
     // two accumulator sets (even / odd code word) halve the MMA dependency chains
     float acc[T][4], acc2[T][4];
 #pragma unroll
@@ -204,20 +243,39 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             acc[n][i] = acc2[n][i] = 0.f;
 
     float *red = reinterpret_cast<float *>(bp + L.red);
-    if (!is_u) {
+    if (producer) {
+        if (lane == 0) {
+            int st = 0;
+            uint32_t prev = 0;   // parity of the stage's previous use
+            for (int c = S; c < nch; ++c) {
+                // stage st is free once every consumer warp has released chunk c - S
+                if (!wait_bounded(bar_empty + 8 * st, prev)) {
+                    atomicOr(p.status, kStatusTimeout);
+                    break;
+                }
+                issue_codes(c, st);
+                issue_x(c, st);
+                issued = c + 1;
+                if (++st == S) {
+                    st = 0;
+                    prev ^= 1u;
+                }
+            }
+        }
+        __syncwarp();
+    } else if (!is_u) {
         // ---- 64 weight rows: warps w and w+4 own rows 16w .. 16w+15, sub-blocks of parity w>>2
         const int kpar = warp >> 2;
         const uint32_t nbg = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + zg_raw)));
         const uint32_t nbh = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + zh_raw)));
         const uint32_t negg = nbg | (nbg << 16), negh = nbh | (nbh << 16);
-        // the codes were requested before the wait for the previous kernel and
-        // have normally landed: one wait for all, so that no compiler barrier
-        // sits inside the loop
-        for (int c = 0; c < nch; ++c)
-            ok = ok && wait_bounded(bar_chunk + 8 * c, 0);
-#pragma unroll 2
-        for (int c = 0; c < (ok ? nch : 0); ++c) {
-            const uint8_t *ctile = bp + L.codes + c * 8192;
+        int s = 0;
+        uint32_t par = 0;
+        for (int c = 0; c < nch && ok; ++c) {
+            ok = wait_bounded(bar_full_w + 8 * s, par) && wait_bounded(bar_full_x + 8 * s, par);
+            if (!ok)
+                break;
+            const uint8_t *ctile = bp + L.ring + s * kStage;
 #pragma unroll
             for (int sb2 = 0; sb2 < 2; ++sb2) {
                 const int sb = 2 * sb2 + kpar;
@@ -225,7 +283,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 const int chunk = ((2 * sb + (cl >> 1)) ^ (rg & 7)) * 16 + (cl & 1) * 8;
                 const uint2 wgv = *reinterpret_cast<const uint2 *>(ctile + rg * 128 + chunk);
                 const uint2 whv = *reinterpret_cast<const uint2 *>(ctile + (rg + 8) * 128 + chunk);
-                const uint8_t *xt = bp + L.x + (4 * c + sb) * (TOK * 128);
+                const uint8_t *xt = ctile + 8192 + sb * (TOK * 128);
                 uint4 xv[T][2];
 #pragma unroll
                 for (int n = 0; n < T; ++n) {
@@ -236,7 +294,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const uint32_t wgw = j ? wgv.y : wgv.x, whw = j ? whv.y : whv.x;
-                    // codes k = 8j + {0..7}: pairs (0,4) (1,5) (2,6) (3,7)
+                    // codes k = 8j + {0..7}: nibbles (m, m + 4) hold the pair k = 2m, 2m + 1,
+                    // the order of the activations in v
                     const uint32_t g0 = dequant_pair(wgw, negg), g1 = dequant_pair(wgw >> 4, negg);
                     const uint32_t g2 = dequant_pair(wgw >> 8, negg), g3 = dequant_pair(wgw >> 12, negg);
                     const uint32_t h0 = dequant_pair(whw, negh), h1 = dequant_pair(whw >> 4, negh);
@@ -244,13 +303,19 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 #pragma unroll
                     for (int n = 0; n < T; ++n) {
                         const uint4 v = xv[n][j];
-                        const uint32_t b0 = prmt(v.x, v.z, 0x5410), b1 = prmt(v.x, v.z, 0x7632);
-                        const uint32_t b2 = prmt(v.y, v.w, 0x5410), b3 = prmt(v.y, v.w, 0x7632);
                         float (&a)[4] = j ? acc2[n] : acc[n];
-                        mma_bf16_16816(a, g0, h0, g1, h1, b0, b1);
-                        mma_bf16_16816(a, g2, h2, g3, h3, b2, b3);
+                        mma_bf16_16816(a, g0, h0, g1, h1, v.x, v.y);
+                        mma_bf16_16816(a, g2, h2, g3, h3, v.z, v.w);
                     }
                 }
+            }
+            // every lane's shared-memory reads of this stage are done: release it
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_empty + 8 * s);
+            if (++s == S) {
+                s = 0;
+                par ^= 1u;
             }
         }
 #pragma unroll
@@ -267,36 +332,46 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             mine[(rg + 8) * TOK + col] = acc[n][2];
             mine[(rg + 8) * TOK + col + 1] = acc[n][3];
         }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < TOK / 4; ++i) {
-            const int e = tid + kThreads * i;   // row e / TOK, token e % TOK
-            red[e] = red[e] + red[kRows * TOK + e];
-        }
     } else {
-        // ---- 16 rows of G = [w_g; A^T]: warp w takes the 64-wide sub-tiles i = w (mod 8)
-        for (int i = warp; i < nsub && ok; i += 8) {
-            ok = wait_bounded(bar_chunk + 8 * (i >> 2), 0);
-            const uint8_t *gt = bp + L.codes + i * 2048;
-            const uint8_t *xt = bp + L.x + i * (TOK * 128);
-            const int ra = gid, rb = gid + 8;
-            const uint4 a0 = *reinterpret_cast<const uint4 *>(gt + ra * 128 + (((2 * cl) ^ (ra & 7)) << 4));
-            const uint4 a1 = *reinterpret_cast<const uint4 *>(gt + ra * 128 + (((2 * cl + 1) ^ (ra & 7)) << 4));
-            const uint4 b0 = *reinterpret_cast<const uint4 *>(gt + rb * 128 + (((2 * cl) ^ (rb & 7)) << 4));
-            const uint4 b1 = *reinterpret_cast<const uint4 *>(gt + rb * 128 + (((2 * cl + 1) ^ (rb & 7)) << 4));
-            const uint32_t ga[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            const uint32_t ha[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        // ---- 16 rows of G = [w_g; A^T]: sub-tile i (64 k, global index 4c + j) is warp i mod 8's
+        int s = 0;
+        uint32_t par = 0;
+        for (int c = 0; c < nch && ok; ++c) {
+            ok = wait_bounded(bar_full_w + 8 * s, par) && wait_bounded(bar_full_x + 8 * s, par);
+            if (!ok)
+                break;
+            const uint8_t *stage = bp + L.ring + s * kStage;
+            for (int j = 0; j < 4; ++j) {
+                if (((4 * c + j) & 7) != warp)
+                    continue;
+                const uint8_t *gt = stage + j * 2048;
+                const uint8_t *xt = stage + 8192 + j * (TOK * 128);
+                const int ra = gid, rb = gid + 8;
+                const uint4 a0 = *reinterpret_cast<const uint4 *>(gt + ra * 128 + (((2 * cl) ^ (ra & 7)) << 4));
+                const uint4 a1 = *reinterpret_cast<const uint4 *>(gt + ra * 128 + (((2 * cl + 1) ^ (ra & 7)) << 4));
+                const uint4 b0 = *reinterpret_cast<const uint4 *>(gt + rb * 128 + (((2 * cl) ^ (rb & 7)) << 4));
+                const uint4 b1 = *reinterpret_cast<const uint4 *>(gt + rb * 128 + (((2 * cl + 1) ^ (rb & 7)) << 4));
+                const uint32_t ga[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const uint32_t ha[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int n = 0; n < T; ++n) {
-                const int t = 8 * n + gid;
-                const uint4 x0 = *reinterpret_cast<const uint4 *>(xt + t * 128 + (((2 * cl) ^ (t & 7)) << 4));
-                const uint4 x1 = *reinterpret_cast<const uint4 *>(xt + t * 128 + (((2 * cl + 1) ^ (t & 7)) << 4));
-                const uint32_t xa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-                // natural pairs: step s covers k = 16 cl + 4s + {0,1} and + {2,3}
+                for (int n = 0; n < T; ++n) {
+                    const int t = 8 * n + gid;
+                    const uint4 x0 = *reinterpret_cast<const uint4 *>(xt + t * 128 + (((2 * cl) ^ (t & 7)) << 4));
+                    const uint4 x1 = *reinterpret_cast<const uint4 *>(xt + t * 128 + (((2 * cl + 1) ^ (t & 7)) << 4));
+                    const uint32_t xa[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                    // natural pairs: step s covers k = 16 cl + 4s + {0,1} and + {2,3}
 #pragma unroll
-                for (int s = 0; s < 4; ++s)
-                    mma_bf16_16816((s & 1) ? acc2[n] : acc[n], ga[2 * s], ha[2 * s], ga[2 * s + 1], ha[2 * s + 1],
-                                   xa[2 * s], xa[2 * s + 1]);
+                    for (int q = 0; q < 4; ++q)
+                        mma_bf16_16816((q & 1) ? acc2[n] : acc[n], ga[2 * q], ha[2 * q], ga[2 * q + 1],
+                                       ha[2 * q + 1], xa[2 * q], xa[2 * q + 1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_empty + 8 * s);
+            if (++s == S) {
+                s = 0;
+                par ^= 1u;
             }
         }
 #pragma unroll
@@ -313,27 +388,41 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             mine[(gid + 8) * TOK + col] = acc[n][2];
             mine[(gid + 8) * TOK + col + 1] = acc[n][3];
         }
-        __syncthreads();
-        for (int e = tid; e < 16 * TOK; e += kThreads) {
-            float s = red[e];
-#pragma unroll
-            for (int w = 1; w < 8; ++w)
-                s += red[w * 16 * TOK + e];
-            red[e] = s;
-        }
     }
     if (!ok)
         atomicOr(p.status, kStatusTimeout);
     __syncthreads();
-    if (tid == 0) {
+    if (tid < kConsumers) {
+        if (!is_u) {
+#pragma unroll
+            for (int i = 0; i < TOK / 4; ++i) {
+                const int e = tid + kConsumers * i;   // row e / TOK, token e % TOK
+                red[e] = red[e] + red[kRows * TOK + e];
+            }
+        } else {
+            for (int e = tid; e < 16 * TOK; e += kConsumers) {
+                float s = red[e];
+#pragma unroll
+                for (int w = 1; w < 8; ++w)
+                    s += red[w * 16 * TOK + e];
+                red[e] = s;
+            }
+        }
+    } else if (lane == 0) {
         // no copy of this CTA may still be landing when it goes on (bounded;
-        // immediate unless a wait above gave up)
-        for (int c = 0; c < nch; ++c)
-            wait_bounded(bar_chunk + 8 * c, 0);
-        wait_bounded(bar_x, 0);
+        // immediate unless a wait gave up): stages reused before the last S
+        // chunks were released by the consumers after they landed
+        for (int c = max(0, issued - S); c < issued; ++c) {
+            wait_bounded(bar_full_w + 8 * (c % S), (uint32_t)(c / S) & 1u);
+            wait_bounded(bar_full_x + 8 * (c % S), (uint32_t)(c / S) & 1u);
+        }
+        for (int c = issued; c < first; ++c)   // codes requested, activations never
+            wait_bounded(bar_full_w + 8 * c, 0);
         if (!is_u && rank == 0 && p.rp > 0)
             wait_bounded(bar_bt, 0);
     }
+    __syncwarp();
+    __syncthreads();
 
     if (is_u) {
         // ---- publish this CTA's partial of u rows 16*cluster .. +15 (all TOK
@@ -352,12 +441,11 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     }
 
     // ---- sum the K split over the cluster, in rank order, in the first CTA.
-    // With an EC, the last warp of the first CTA meanwhile waits until u is
-    // published.
+    // With an EC, the last consumer warp of the first CTA meanwhile waits until
+    // u is published; the producer warp only takes part in the barriers.
     const bool ec_warp = rank == 0 && p.JB > 0 && warp == kEcWarp;
-    const int nsum = p.JB > 0 ? kThreads - 32 : kThreads;
+    const int nsum = p.JB > 0 ? kConsumers - 32 : kConsumers;   // summing threads: tid < nsum
     constexpr int tile4 = kRows * TOK / 4;
-    __shared__ int s_good;
     if (push) {
         cluster_wait();   // every receive barrier of the cluster is initialised
         if (rank != 0) {
@@ -375,9 +463,10 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         } else if (CS > 1 && !wait_bounded(bar_recv, 0) && tid == 0) {
             atomicOr(p.status, kStatusTimeout);
         }
+        __syncwarp();
         cluster_arrive();     // the tiles have landed: the other CTAs may leave
         const float4 *slots = reinterpret_cast<const float4 *>(bp + L.recv);
-        if (!ec_warp)
+        if (tid < nsum)
             for (int e4 = tid; e4 < tile4; e4 += nsum) {
                 float4 s = reinterpret_cast<const float4 *>(red)[e4];
                 for (int q = 0; q < CS - 1; ++q) {
@@ -390,12 +479,11 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 reinterpret_cast<float4 *>(red)[e4] = s;
             }
     } else {
-        __syncthreads();
         cluster_sync();
         if (ec_warp) {
             if (lane == 0)
                 s_good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
-        } else if (rank == 0) {
+        } else if (rank == 0 && tid < nsum) {
             const uint32_t red_addr = base + L.red;
             for (int e4 = tid; e4 < tile4; e4 += nsum) {
                 // issue every remote load before summing (in rank order)
@@ -416,6 +504,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 reinterpret_cast<float4 *>(red)[e4] = s;
             }
         }
+        __syncwarp();
         cluster_sync();  // the other CTAs' shared memory is no longer read
         if (rank != 0)
             return;
@@ -456,80 +545,102 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         }
     }
 
-    // ---- epilogue of a 64-row cluster
-    if (p.JB > 0 && !wait_bounded(bar_bt, 0))
-        atomicOr(p.status, kStatusTimeout);
-    const int row = tid & (kRows - 1), th = tid >> 6;  // four token phases
-    const int64_t n = n0 + row;
-    float out[TOK / 4];
-#pragma unroll
-    for (int i = 0; i < TOK / 4; ++i)
-        out[i] = s_epi * red[row * TOK + th + 4 * i];
-    if (p.JB > 0) {
-        // corr = g_t * sum_j u[1 + j][t] * B^T[n][j]: the B^T row in 16-byte pieces,
-        // u broadcast, both from shared memory
-        float corr[TOK / 4];
+    // ---- epilogue of a 64-row cluster (consumer threads: 64 rows x 4 token phases)
+    if (tid < kConsumers) {
+        if (p.JB > 0 && !wait_bounded(bar_bt, 0))
+            atomicOr(p.status, kStatusTimeout);
+        const int row = tid & (kRows - 1), th = tid >> 6;
+        const int64_t n = n0 + row;
+        float out[TOK / 4];
 #pragma unroll
         for (int i = 0; i < TOK / 4; ++i)
-            corr[i] = 0.f;
-        const uint16_t *btrow = reinterpret_cast<const uint16_t *>(bp + L.bt) + row * p.rp;
-        for (int j0 = 0; j0 < p.rp; j0 += 8) {
-            const uint4 bv = *reinterpret_cast<const uint4 *>(btrow + j0);
-            const float bj[8] = {bf16_lo(bv.x), bf16_hi(bv.x), bf16_lo(bv.y), bf16_hi(bv.y),
-                                 bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
+            out[i] = s_epi * red[row * TOK + th + 4 * i];
+        if (p.JB > 0) {
+            // corr = g_t * sum_j u[1 + j][t] * B^T[n][j]: the B^T row in 16-byte pieces,
+            // u broadcast, both from shared memory
+            float corr[TOK / 4];
+#pragma unroll
+            for (int i = 0; i < TOK / 4; ++i)
+                corr[i] = 0.f;
+            const uint16_t *btrow = reinterpret_cast<const uint16_t *>(bp + L.bt) + row * p.rp;
+            for (int j0 = 0; j0 < p.rp; j0 += 8) {
+                const uint4 bv = *reinterpret_cast<const uint4 *>(btrow + j0);
+                const float bj[8] = {bf16_lo(bv.x), bf16_hi(bv.x), bf16_lo(bv.y), bf16_hi(bv.y),
+                                     bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
+#pragma unroll
+                for (int i = 0; i < TOK / 4; ++i) {
+                    const float4 *ut = reinterpret_cast<const float4 *>(uT + (th + 4 * i) * p.rp + j0);
+                    const float4 v0 = ut[0], v1 = ut[1];
+                    corr[i] += v0.x * bj[0] + v0.y * bj[1] + v0.z * bj[2] + v0.w * bj[3] + v1.x * bj[4] +
+                               v1.y * bj[5] + v1.z * bj[6] + v1.w * bj[7];
+                }
+            }
 #pragma unroll
             for (int i = 0; i < TOK / 4; ++i) {
-                const float4 *ut = reinterpret_cast<const float4 *>(uT + (th + 4 * i) * p.rp + j0);
-                const float4 v0 = ut[0], v1 = ut[1];
-                corr[i] += v0.x * bj[0] + v0.y * bj[1] + v0.z * bj[2] + v0.w * bj[3] + v1.x * bj[4] +
-                           v1.y * bj[5] + v1.z * bj[6] + v1.w * bj[7];
+                const float g = 1.0f / (1.0f + expf(-(u0[th + 4 * i] + p.b_g)));
+                out[i] += g * corr[i];
             }
         }
 #pragma unroll
         for (int i = 0; i < TOK / 4; ++i) {
-            const float g = 1.0f / (1.0f + expf(-(u0[th + 4 * i] + p.b_g)));
-            out[i] += g * corr[i];
+            const int t = th + 4 * i;
+            if (t < p.M && n < p.N)
+                p.y[(int64_t)t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
         }
-    }
-#pragma unroll
-    for (int i = 0; i < TOK / 4; ++i) {
-        const int t = th + 4 * i;
-        if (t < p.M && n < p.N)
-            p.y[(int64_t)t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
     }
     if (push)
         cluster_wait();
 }
 
-// Cluster size CS (CTAs splitting K) and the k per CTA, or 0 if a slice would
-// not fit in shared memory.  Preferably the grid takes about two CTAs per SM,
-// so that the next layer's kernel (launched early) finds room to start its
-// weight copies while this one runs; layers too large for that take up to 8
-// CTAs per SM.  No rank is left without a chunk.
+// Cluster size CS (CTAs splitting K) and the k per CTA: the largest CS (at
+// most 8) whose grid is one wave of two CTAs per SM (so that the next
+// layer's kernel, launched early, also finds room), else CS = 1.  No rank is
+// left without a chunk.  The slice is streamed, so its length is not bounded.
 int pick_cluster(const Packed &pk, int num_sms, int JB, int *KS_out)
 {
     const int NC = (int)(pk.Np / kRows);
     const int chunks = (int)(pk.Kp / kChunk);
-    for (int limit : {2, 8}) {
-        for (int CS = std::min(8, chunks); CS >= 1; --CS) {
-            const int per = (chunks + CS - 1) / CS;
-            if (per > kMaxChunks || (CS - 1) * per >= chunks)
-                continue;
-            if ((int64_t)(NC + JB) * CS <= (int64_t)limit * num_sms) {
-                *KS_out = per * kChunk;
-                return CS;
-            }
-        }
-    }
-    // otherwise the fewest chunks per CTA that fit
     for (int CS = std::min(8, chunks); CS >= 1; --CS) {
         const int per = (chunks + CS - 1) / CS;
-        if (per <= kMaxChunks && (CS == 1 || (CS - 1) * per < chunks)) {
+        if (CS > 1 && (CS - 1) * per >= chunks)
+            continue;
+        if (CS == 1 || (int64_t)(NC + JB) * CS <= 2LL * num_sms) {
             *KS_out = per * kChunk;
             return CS;
         }
     }
     return 0;
+}
+
+// Ring depth: as many stages as fit in the per-CTA budget beside the other
+// regions, at most the chunks of the slice, and two when the slice has two
+// chunks or more (then the budget may be exceeded).
+template <int TOK>
+int pick_stages(int nch, int rp, int nslots)
+{
+    const int fixed = (int)smem_layout<TOK>(0, rp, nslots).total + 1024;
+    const int fit = (kSmemPerCta - fixed) / (int)stage_bytes<TOK>();
+    return std::max(std::min(2, nch), std::min({fit, nch, kMaxStages}));
+}
+
+struct Plan {
+    int S, push;
+    size_t smem;
+};
+
+template <int TOK>
+Plan plan_for(int nch, int rp, int CS)
+{
+    Plan pl;
+    // push the partial tiles when the receive slots fit, else pull them over DSMEM
+    pl.S = pick_stages<TOK>(nch, rp, CS - 1);
+    pl.smem = smem_layout<TOK>(pl.S, rp, CS - 1).total + 1024;
+    pl.push = pl.smem <= 227 * 1024 ? 1 : 0;
+    if (!pl.push) {
+        pl.S = pick_stages<TOK>(nch, rp, 0);
+        pl.smem = smem_layout<TOK>(pl.S, rp, 0).total + 1024;
+    }
+    return pl;
 }
 
 template <int T>
@@ -548,7 +659,7 @@ bool decode_supported(const Packed &pk, int num_sms)
     const int CS = pick_cluster(pk, num_sms, pk.r > 0 ? pk.R1p / 16 : 0, &KS);
     if (CS == 0)
         return false;
-    return smem_layout<32>(KS, pk.rp, pk.R1p, 0).total + 1024 <= 227 * 1024;
+    return plan_for<32>(KS / kChunk, pk.rp, CS).smem <= 227 * 1024;
 }
 
 cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
@@ -628,23 +739,21 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
                              (uint32_t)(8 * T), CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess)
         return e;
-    // push the partial tiles when the receive slots fit, else pull them over DSMEM
-    auto layout = [&](int nslots) {
-        return T == 1 ? smem_layout<8>(p.KS, p.rp, p.R1p, nslots)
-                      : (T == 2 ? smem_layout<16>(p.KS, p.rp, p.R1p, nslots)
-                                : smem_layout<32>(p.KS, p.rp, p.R1p, nslots));
-    };
-    p.push = layout(CS - 1).total + 1024 <= 227 * 1024 ? 1 : 0;
-    const size_t smem = layout(p.push ? CS - 1 : 0).total + 1024;
+    const Plan pl = T == 1 ? plan_for<8>(p.nch, p.rp, CS)
+                           : (T == 2 ? plan_for<16>(p.nch, p.rp, CS) : plan_for<32>(p.nch, p.rp, CS));
+    if (pl.smem > 227 * 1024)
+        return cudaErrorInvalidValue;
+    p.S = pl.S;
+    p.push = pl.push;
     const void *fn = T == 1 ? kernel_ptr<1>() : (T == 2 ? kernel_ptr<2>() : kernel_ptr<4>());
-    e = raise_smem_limit(fn, smem);
+    e = raise_smem_limit(fn, pl.smem);
     if (e != cudaSuccess)
         return e;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((p.JB + p.NC) * CS));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -31,6 +31,13 @@ __device__ __forceinline__ uint32_t fma_bf16x2(uint32_t a, uint32_t b, uint32_t 
     return d;
 }
 
+// Stored nibble order of a code word (the tiled layout on the device): the
+// codes of k = 8j + {0, 2, 4, 6} sit in nibbles 0..3 and those of k = 8j +
+// {1, 3, 5, 7} in nibbles 4..7, so that the nibble pair (m, m + 4), 16 bits
+// apart, is the consecutive pair k = 8j + 2m, 8j + 2m + 1.  Bit offset of the
+// code of k = 8j + i:
+__host__ __device__ constexpr int nibble_shift(int i) { return 4 * ((i & 1) * 4 + (i >> 1)); }
+
 // Two int4 codes, the nibbles at bit positions `sh` and `sh + 16` of w, as a
 // bf16x2 pair of exact integers (q_lo - zp, q_hi - zp).  The nibble is placed
 // in the low mantissa bits of 128.0 (0x4300), giving 128 + q exactly; the fma

@@ -11,7 +11,8 @@ cudaError_t raise_smem_limit(const void *func, size_t bytes);
 
 // Library-owned packed layout (all device memory, zero/neutral padded):
 //   codes tiled [Np/64][Kp/256][64][32] uint32: the word holding codes k = 8j..8j+7
-//                             of row n (code of k = 8j+i in bits [4i,4i+3]) sits at
+//                             of row n (code of k = 8j+i at bit nibble_shift(i), i.e.
+//                             even k in nibbles 0..3, odd k in nibbles 4..7) sits at
 //                             ((n/64 * Kp/256 + j/32) * 64 + n%64) * 32 + j%32, so every
 //                             64-row x 256-k block is 8 KB of contiguous memory;
 //                             padding words hold code 8 (weight 0)

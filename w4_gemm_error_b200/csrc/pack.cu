@@ -8,9 +8,11 @@
 //   s[n] = fp32(max_k |W[n,k]|) / 7        (IEEE fp32 division)
 //   q    = clamp(rint(fp32(W[n,k] / s[n])), -8, 7) + 8    (ties to even)
 //   z[n] = 8;  an all-zero row has s = 0 and every code 8
-//   code of k = 8j+i in bits [4i, 4i+3] of word j of row n (exported
-//   layout [N][K/8]; stored tiled in 8 KB blocks of 64 rows x 256 k, see
-//   kernels.h).
+//   code of k = 8j+i in bits [4i, 4i+3] of word j of row n in the exported
+//   layout [N][K/8]; on the device the words are stored tiled in 8 KB blocks
+//   of 64 rows x 256 k (see kernels.h) with their nibbles in the order of
+//   nibble_shift (device_utils.cuh), which the dequantisers unpack as
+//   consecutive k pairs.
 #include "device_utils.cuh"
 #include "kernels.h"
 
@@ -74,7 +76,7 @@ pack_w4_kernel(const uint16_t *__restrict__ W, int64_t N, int64_t K, int64_t Np,
                 const uint32_t h = (i & 1) ? (w4[i >> 1] & 0xFFFF0000u) : (w4[i >> 1] << 16);
                 float c = rintf(__fdiv_rn(__uint_as_float(h), sn));
                 c = fminf(fmaxf(c, -8.0f), 7.0f);
-                word |= (uint32_t)((int)c + 8) << (4 * i);
+                word |= (uint32_t)((int)c + 8) << nibble_shift(i);
             }
         }
         word_at(j) = word;
@@ -119,6 +121,16 @@ __global__ void pack_ec_kernel(const uint16_t *__restrict__ A, const uint16_t *_
     }
 }
 
+// Back to the documented order: code of k = 8j + i in bits [4i, 4i + 3].
+__device__ __forceinline__ uint32_t natural_nibble_order(uint32_t w)
+{
+    uint32_t out = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        out |= ((w >> nibble_shift(i)) & 0xFu) << (4 * i);
+    return out;
+}
+
 __global__ void untile_codes_kernel(const uint32_t *__restrict__ tiled, uint32_t *__restrict__ dst, int64_t N,
                                     int64_t K, int64_t Kp)
 {
@@ -126,7 +138,7 @@ __global__ void untile_codes_kernel(const uint32_t *__restrict__ tiled, uint32_t
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < N * words;
          i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t n = i / words, j = i - n * words;
-        dst[i] = tiled[(((n >> 6) * (Kp / 256) + (j >> 5)) * 64 + (n & 63)) * 32 + (j & 31)];
+        dst[i] = natural_nibble_order(tiled[(((n >> 6) * (Kp / 256) + (j >> 5)) * 64 + (n & 63)) * 32 + (j & 31)]);
     }
 }
 

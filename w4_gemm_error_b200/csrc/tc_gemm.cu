@@ -382,14 +382,12 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 #pragma unroll
                     for (int jj = 0; jj < 4; ++jj) {
                         const int j = 4 * half + jj;
-                        // codes k = 8j + {0..7}: pairs (0,4) (1,5) (2,6) (3,7)
-                        const uint32_t p0 = dequant_pair(words[jj], negz), p1 = dequant_pair(words[jj] >> 4, negz);
-                        const uint32_t p2 = dequant_pair(words[jj] >> 8, negz), p3 = dequant_pair(words[jj] >> 12, negz);
+                        // codes k = 8j + {0..7}: nibbles (m, m + 4) hold k = 2m, 2m + 1
                         uint4 o;
-                        o.x = prmt(p0, p1, 0x5410);   // k 0, 1
-                        o.y = prmt(p2, p3, 0x5410);   // k 2, 3
-                        o.z = prmt(p0, p1, 0x7632);   // k 4, 5
-                        o.w = prmt(p2, p3, 0x7632);   // k 6, 7
+                        o.x = dequant_pair(words[jj], negz);         // k 0, 1
+                        o.y = dequant_pair(words[jj] >> 4, negz);    // k 2, 3
+                        o.z = dequant_pair(words[jj] >> 8, negz);    // k 4, 5
+                        o.w = dequant_pair(words[jj] >> 12, negz);   // k 6, 7
                         *reinterpret_cast<uint4 *>(arow + ((j ^ (i & 7)) << 4)) = o;
                     }
                     fence_proxy_async_smem();
