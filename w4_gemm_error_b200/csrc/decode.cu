@@ -17,8 +17,9 @@
 //    short slice is then entirely resident), and the consumers sleep in a CTA
 //    barrier until the activations are on their way;
 //  * eight consumer warps, two per 16-row group splitting the 64-wide
-//    sub-blocks of each stage, so the dequantise-MMA chains of one warp hide
-//    another's;
+//    sub-blocks of each stage, or, for one token group on a short slice,
+//    sixteen (one per 16-row group and sub-block), so the dequantise-MMA
+//    chains of one warp hide another's;
 //  * weight rows sit on the 16-row side of mma.sync m16n8k16 and tokens on
 //    the 8-column side, so a code is read once for up to 32 tokens; the
 //    codes are dequantised in registers to exact (q - z) bf16 pairs (two
@@ -57,10 +58,9 @@ constexpr int kRows = 64;         // weight rows per cluster (four warps x 16)
 constexpr int kChunk = 256;       // k per stage (one 8 KB TMA box of 64 rows of codes)
 constexpr int kMaxStages = 8;     // ring depth limit
 constexpr int kUStride = 32;      // token stride of the published u rows
-constexpr int kConsumers = 256;   // 8 consumer warps: two per 16-row group
-constexpr int kThreads = kConsumers + 32;   // + one producer warp
-constexpr int kProducerWarp = kConsumers / 32;
-constexpr int kEcWarp = kProducerWarp - 1;  // consumer warp that waits for u
+// A CTA has W consumer warps, W = 16 (one per 16-row group and 64-k
+// sub-block of a stage) or W = 8 (two sub-blocks each), then one producer warp.
+__host__ __device__ constexpr int block_threads(int W) { return 32 * W + 32; }
 // shared memory per CTA that keeps two CTAs per SM resident
 constexpr int kSmemPerCta = 110 * 1024;
 
@@ -101,15 +101,16 @@ struct Smem {
     uint32_t total;
 };
 
-// S ring stages; nslots receive slots of one partial tile (64 rows x TOK fp32) each.
+// S ring stages; W consumer warps; nslots receive slots of one partial tile
+// (64 rows x TOK fp32) each.
 template <int TOK>
-__host__ __device__ inline Smem smem_layout(int S, int rp, int nslots)
+__host__ __device__ inline Smem smem_layout(int S, int rp, int nslots, int W)
 {
     Smem m;
     m.ring = 0;
     m.bt = m.ring + S * stage_bytes<TOK>();        // 128*rp bytes: B^T rows of the cluster
-    m.red = m.bt + 128 * rp;                       // 512*TOK bytes: partial tiles
-    m.u = m.red + 512 * TOK;                       // u0 [TOK], uT [TOK][rp] (fp32)
+    m.red = m.bt + 128 * rp;                       // partial tiles: 64*W*TOK bytes
+    m.u = m.red + 64 * W * TOK;                    // u0 [TOK], uT [TOK][rp] (fp32)
     m.recv = (m.u + 4 * TOK * (rp + 1) + 15) & ~15u;
     m.total = m.recv + nslots * 256 * TOK;
     return m;
@@ -132,15 +133,21 @@ __device__ __forceinline__ bool wait_u_published(const DecodeParams &p, unsigned
     return true;
 }
 
-// Register budget: three CTAs per SM up to 16 tokens (the grid is about two
-// per SM, and the next layer's kernel starts beside it), two at 32 tokens.
-template <int T>
-__global__ void __launch_bounds__(kThreads, T == 4 ? 2 : 3)
+// Register budget: with 16 consumer warps two CTAs per SM; with 8, three
+// CTAs per SM up to 16 tokens (the grid is about two per SM, and the next
+// layer's kernel starts beside it) and two at 32 tokens.
+template <int T, int W>
+__global__ void __launch_bounds__(block_threads(W), (W == 16 || T == 4) ? 2 : 3)
 decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_g,
                    const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_x,
                    DecodeParams p, int CS)
 {
     constexpr int TOK = 8 * T;
+    constexpr int kConsumers = 32 * W;
+    constexpr int kThreads = block_threads(W);
+    constexpr int kProducerWarp = W;
+    constexpr int kEcWarp = W - 1;   // consumer warp that waits for u
+    constexpr int KPAR = W / 4;      // consumer warps per 16-row group
     constexpr uint32_t kStage = stage_bytes<TOK>();
     constexpr uint32_t kXBytes = 4 * TOK * 128;
     extern __shared__ uint8_t smem_raw[];
@@ -155,7 +162,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const bp = smem_raw + (base - raw);
     const bool push = p.push != 0;
-    const Smem L = smem_layout<TOK>(p.S, p.rp, push ? CS - 1 : 0);
+    const Smem L = smem_layout<TOK>(p.S, p.rp, push ? CS - 1 : 0, W);
     const uint32_t rank = cluster_ctarank();
     const int cluster = blockIdx.x / CS;
     const bool is_u = cluster < p.JB;
@@ -202,7 +209,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         for (int i = 0; i < kMaxStages; ++i) {
             mbar_init(bar_full_w + 8 * i, 1);
             mbar_init(bar_full_x + 8 * i, 1);
-            mbar_init(bar_empty + 8 * i, kConsumers / 32);
+            mbar_init(bar_empty + 8 * i, W);
         }
         mbar_init(bar_bt, 1);
         mbar_init(bar_recv, 1);
@@ -264,8 +271,9 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         }
         __syncwarp();
     } else if (!is_u) {
-        // ---- 64 weight rows: warps w and w+4 own rows 16w .. 16w+15, sub-blocks of parity w>>2
-        const int kpar = warp >> 2;
+        // ---- 64 weight rows: warp w owns rows 16(w mod 4) .. +15 and the sub-blocks
+        // sb = w/4 (mod KPAR) of each stage
+        const int kq = warp >> 2;
         const uint32_t nbg = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + zg_raw)));
         const uint32_t nbh = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + zh_raw)));
         const uint32_t negg = nbg | (nbg << 16), negh = nbh | (nbh << 16);
@@ -277,8 +285,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 break;
             const uint8_t *ctile = bp + L.ring + s * kStage;
 #pragma unroll
-            for (int sb2 = 0; sb2 < 2; ++sb2) {
-                const int sb = 2 * sb2 + kpar;
+            for (int i = 0; i < 4 / KPAR; ++i) {
+                const int sb = KPAR * i + kq;
                 // codes k = 64 sb + 16 cl + {0..15} of rows rg and rg + 8 (8 bytes each)
                 const int chunk = ((2 * sb + (cl >> 1)) ^ (rg & 7)) * 16 + (cl & 1) * 8;
                 const uint2 wgv = *reinterpret_cast<const uint2 *>(ctile + rg * 128 + chunk);
@@ -323,7 +331,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 acc[n][i] += acc2[n][i];
-        float *mine = red + kpar * kRows * TOK;   // [2][64][TOK]
+        float *mine = red + kq * kRows * TOK;   // [KPAR][64][TOK]
 #pragma unroll
         for (int n = 0; n < T; ++n) {
             const int col = 8 * n + 2 * cl;
@@ -333,7 +341,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             mine[(rg + 8) * TOK + col + 1] = acc[n][3];
         }
     } else {
-        // ---- 16 rows of G = [w_g; A^T]: sub-tile i (64 k, global index 4c + j) is warp i mod 8's
+        // ---- 16 rows of G = [w_g; A^T]: sub-tile i (64 k, global index 4c + j) is warp (i mod W)'s
         int s = 0;
         uint32_t par = 0;
         for (int c = 0; c < nch && ok; ++c) {
@@ -342,7 +350,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 break;
             const uint8_t *stage = bp + L.ring + s * kStage;
             for (int j = 0; j < 4; ++j) {
-                if (((4 * c + j) & 7) != warp)
+                if ((4 * c + j) % W != warp)
                     continue;
                 const uint8_t *gt = stage + j * 2048;
                 const uint8_t *xt = stage + 8192 + j * (TOK * 128);
@@ -379,7 +387,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 acc[n][i] += acc2[n][i];
-        float *mine = red + warp * 16 * TOK;  // [8 warps][16][TOK]
+        float *mine = red + warp * 16 * TOK;  // [W][16][TOK]
 #pragma unroll
         for (int n = 0; n < T; ++n) {
             const int col = 8 * n + 2 * cl;
@@ -394,16 +402,18 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     __syncthreads();
     if (tid < kConsumers) {
         if (!is_u) {
+            for (int e = tid; e < kRows * TOK; e += kConsumers) {   // row e / TOK, token e % TOK
+                float s = red[e];
 #pragma unroll
-            for (int i = 0; i < TOK / 4; ++i) {
-                const int e = tid + kConsumers * i;   // row e / TOK, token e % TOK
-                red[e] = red[e] + red[kRows * TOK + e];
+                for (int q = 1; q < KPAR; ++q)
+                    s += red[q * kRows * TOK + e];
+                red[e] = s;
             }
         } else {
             for (int e = tid; e < 16 * TOK; e += kConsumers) {
                 float s = red[e];
 #pragma unroll
-                for (int w = 1; w < 8; ++w)
+                for (int w = 1; w < W; ++w)
                     s += red[w * 16 * TOK + e];
                 red[e] = s;
             }
@@ -545,8 +555,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         }
     }
 
-    // ---- epilogue of a 64-row cluster (consumer threads: 64 rows x 4 token phases)
-    if (tid < kConsumers) {
+    // ---- epilogue of a 64-row cluster (256 threads: 64 rows x 4 token phases)
+    if (tid < 256) {
         if (p.JB > 0 && !wait_bounded(bar_bt, 0))
             atomicOr(p.status, kStatusTimeout);
         const int row = tid & (kRows - 1), th = tid >> 6;
@@ -616,9 +626,9 @@ int pick_cluster(const Packed &pk, int num_sms, int JB, int *KS_out)
 // regions, at most the chunks of the slice, and two when the slice has two
 // chunks or more (then the budget may be exceeded).
 template <int TOK>
-int pick_stages(int nch, int rp, int nslots)
+int pick_stages(int nch, int rp, int nslots, int W)
 {
-    const int fixed = (int)smem_layout<TOK>(0, rp, nslots).total + 1024;
+    const int fixed = (int)smem_layout<TOK>(0, rp, nslots, W).total + 1024;
     const int fit = (kSmemPerCta - fixed) / (int)stage_bytes<TOK>();
     return std::max(std::min(2, nch), std::min({fit, nch, kMaxStages}));
 }
@@ -629,24 +639,29 @@ struct Plan {
 };
 
 template <int TOK>
-Plan plan_for(int nch, int rp, int CS)
+Plan plan_for(int nch, int rp, int CS, int W)
 {
     Plan pl;
     // push the partial tiles when the receive slots fit, else pull them over DSMEM
-    pl.S = pick_stages<TOK>(nch, rp, CS - 1);
-    pl.smem = smem_layout<TOK>(pl.S, rp, CS - 1).total + 1024;
+    pl.S = pick_stages<TOK>(nch, rp, CS - 1, W);
+    pl.smem = smem_layout<TOK>(pl.S, rp, CS - 1, W).total + 1024;
     pl.push = pl.smem <= 227 * 1024 ? 1 : 0;
     if (!pl.push) {
-        pl.S = pick_stages<TOK>(nch, rp, 0);
-        pl.smem = smem_layout<TOK>(pl.S, rp, 0).total + 1024;
+        pl.S = pick_stages<TOK>(nch, rp, 0, W);
+        pl.smem = smem_layout<TOK>(pl.S, rp, 0, W).total + 1024;
     }
     return pl;
 }
 
-template <int T>
+// Consumer warps: 16 for one token group on a short slice (at most four
+// chunks, where hiding latency matters most), else 8, whose per-chunk
+// overhead is shared by two sub-blocks.
+int pick_warps(int T, int nch) { return (T == 1 && nch <= 4) ? 16 : 8; }
+
+template <int T, int W>
 const void *kernel_ptr()
 {
-    return reinterpret_cast<const void *>(decode_w4ec_kernel<T>);
+    return reinterpret_cast<const void *>(decode_w4ec_kernel<T, W>);
 }
 
 }  // namespace
@@ -659,7 +674,7 @@ bool decode_supported(const Packed &pk, int num_sms)
     const int CS = pick_cluster(pk, num_sms, pk.r > 0 ? pk.R1p / 16 : 0, &KS);
     if (CS == 0)
         return false;
-    return plan_for<32>(KS / kChunk, pk.rp, CS).smem <= 227 * 1024;
+    return plan_for<32>(KS / kChunk, pk.rp, CS, 8).smem <= 227 * 1024;
 }
 
 cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
@@ -739,20 +754,22 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
                              (uint32_t)(8 * T), CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess)
         return e;
-    const Plan pl = T == 1 ? plan_for<8>(p.nch, p.rp, CS)
-                           : (T == 2 ? plan_for<16>(p.nch, p.rp, CS) : plan_for<32>(p.nch, p.rp, CS));
+    const int W = pick_warps(T, p.nch);
+    const Plan pl = T == 1 ? plan_for<8>(p.nch, p.rp, CS, W)
+                           : (T == 2 ? plan_for<16>(p.nch, p.rp, CS, W) : plan_for<32>(p.nch, p.rp, CS, W));
     if (pl.smem > 227 * 1024)
         return cudaErrorInvalidValue;
     p.S = pl.S;
     p.push = pl.push;
-    const void *fn = T == 1 ? kernel_ptr<1>() : (T == 2 ? kernel_ptr<2>() : kernel_ptr<4>());
+    const void *fn = T == 1 ? (W == 16 ? kernel_ptr<1, 16>() : kernel_ptr<1, 8>())
+                            : (T == 2 ? kernel_ptr<2, 8>() : kernel_ptr<4, 8>());
     e = raise_smem_limit(fn, pl.smem);
     if (e != cudaSuccess)
         return e;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((p.JB + p.NC) * CS));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3((unsigned)block_threads(W));
     cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -765,9 +782,12 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     switch (T) {
-    case 1: return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<1>, m->codes, m->g, m->bt, tm_x, p, CS);
-    case 2: return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<2>, m->codes, m->g, m->bt, tm_x, p, CS);
-    default: return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<4>, m->codes, m->g, m->bt, tm_x, p, CS);
+    case 1:
+        if (W == 16)
+            return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<1, 16>, m->codes, m->g, m->bt, tm_x, p, CS);
+        return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<1, 8>, m->codes, m->g, m->bt, tm_x, p, CS);
+    case 2: return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<2, 8>, m->codes, m->g, m->bt, tm_x, p, CS);
+    default: return cudaLaunchKernelEx(&cfg, decode_w4ec_kernel<4, 8>, m->codes, m->g, m->bt, tm_x, p, CS);
     }
 }
 
