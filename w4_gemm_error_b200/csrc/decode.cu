@@ -146,14 +146,12 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     constexpr int kConsumers = 32 * W;
     constexpr int kThreads = block_threads(W);
     constexpr int kProducerWarp = W;
-    constexpr int kEcWarp = W - 1;   // consumer warp that waits for u
     constexpr int KPAR = W / 4;      // consumer warps per 16-row group
     constexpr uint32_t kStage = stage_bytes<TOK>();
     constexpr uint32_t kXBytes = 4 * TOK * 128;
     extern __shared__ uint8_t smem_raw[];
     // per stage: codes landed, activations landed, stage free; then B^T, K-split receive
     __shared__ __align__(8) uint64_t bars[3 * kMaxStages + 2];
-    __shared__ int s_good;
 
     pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, cl = lane & 3;
@@ -451,11 +449,45 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     }
 
     // ---- sum the K split over the cluster, in rank order, in the first CTA.
-    // With an EC, the last consumer warp of the first CTA meanwhile waits until
-    // u is published; the producer warp only takes part in the barriers.
-    const bool ec_warp = rank == 0 && p.JB > 0 && warp == kEcWarp;
-    const int nsum = p.JB > 0 ? kConsumers - 32 : kConsumers;   // summing threads: tid < nsum
+    // With an EC, u is published by the EC clusters as CS partials, which are
+    // summed (rank order) into u0 [TOK] (gate logits) and uT [TOK][rp]
+    // (u[1 + j][t] transposed, zero for j >= r): with 16 consumer warps, warps
+    // 0-3 sum the K split while the other twelve wait for u and fetch it; with
+    // 8, the last consumer warp waits for u during the sum and every consumer
+    // thread fetches it afterwards (a fetch by half of the threads needs more
+    // round trips than the overlap saves).  The producer warp only takes part
+    // in the barriers.
+    constexpr bool kOverlap = W == 16;
+    constexpr int kSumThreads = kOverlap ? 128 : kConsumers - 32;
+    const bool fetcher = kOverlap && rank == 0 && p.JB > 0 && tid >= kSumThreads && tid < kConsumers;
+    const bool poller = !kOverlap && rank == 0 && p.JB > 0 && warp == W - 1;
+    const int nsum = p.JB > 0 ? kSumThreads : kConsumers;   // summing threads: tid < nsum
+    __shared__ int s_good;
     constexpr int tile4 = kRows * TOK / 4;
+    float *u0 = reinterpret_cast<float *>(bp + L.u);
+    float *uT = u0 + TOK;
+    auto fetch_u = [&](int ft, int nft, bool good) {
+        for (int e = ft; e < (1 + p.r) * TOK; e += nft) {
+            const int row = e / TOK, t = e - row * TOK;
+            float v[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                v[q] = (q < CS && good) ? __ldcg(p.ws_u + ((int64_t)q * p.R1p + row) * kUStride + t) : 0.f;
+            float u = v[0];
+#pragma unroll
+            for (int q = 1; q < 8; ++q)
+                if (q < CS)
+                    u += v[q];
+            if (row == 0)
+                u0[t] = u;
+            else
+                uT[t * p.rp + row - 1] = u;
+        }
+        for (int e = ft; e < TOK * (p.rp - p.r); e += nft) {
+            const int t = e / (p.rp - p.r), j = p.r + e - t * (p.rp - p.r);
+            uT[t * p.rp + j] = 0.f;
+        }
+    };
     if (push) {
         cluster_wait();   // every receive barrier of the cluster is initialised
         if (rank != 0) {
@@ -467,14 +499,19 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             cluster_wait();   // the first CTA has received every tile
             return;
         }
-        if (ec_warp) {
-            if (lane == 0)
-                s_good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
-        } else if (CS > 1 && !wait_bounded(bar_recv, 0) && tid == 0) {
+        if (!fetcher && !poller && CS > 1 && !wait_bounded(bar_recv, 0) && tid == 0)
             atomicOr(p.status, kStatusTimeout);
-        }
-        __syncwarp();
         cluster_arrive();     // the tiles have landed: the other CTAs may leave
+        if (fetcher || poller) {
+            int good = 1;
+            if (lane == 0)
+                good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
+            good = __shfl_sync(0xffffffffu, good, 0);
+            if (fetcher)
+                fetch_u(tid - kSumThreads, kConsumers - kSumThreads, good != 0);
+            else if (lane == 0)
+                s_good = good;
+        }
         const float4 *slots = reinterpret_cast<const float4 *>(bp + L.recv);
         if (tid < nsum)
             for (int e4 = tid; e4 < tile4; e4 += nsum) {
@@ -490,9 +527,15 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             }
     } else {
         cluster_sync();
-        if (ec_warp) {
+        if (fetcher || poller) {
+            int good = 1;
             if (lane == 0)
-                s_good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
+                good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
+            good = __shfl_sync(0xffffffffu, good, 0);
+            if (fetcher)
+                fetch_u(tid - kSumThreads, kConsumers - kSumThreads, good != 0);
+            else if (lane == 0)
+                s_good = good;
         } else if (rank == 0 && tid < nsum) {
             const uint32_t red_addr = base + L.red;
             for (int e4 = tid; e4 < tile4; e4 += nsum) {
@@ -520,80 +563,66 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             return;
     }
     __syncthreads();
-
-    // ---- EC: u = sum over the CS published partials (rank order), as u0 [TOK]
-    // (gate logits) and uT [TOK][rp] (u[1 + j][t] transposed, zero for j >= r)
-    float *u0 = reinterpret_cast<float *>(bp + L.u);
-    float *uT = u0 + TOK;
-    if (p.JB > 0) {
-        const bool good = s_good != 0;
-        for (int e = tid; e < (1 + p.r) * TOK; e += kThreads) {
-            const int row = e / TOK, t = e - row * TOK;
-            float v[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                v[q] = (q < CS && good) ? __ldcg(p.ws_u + ((int64_t)q * p.R1p + row) * kUStride + t) : 0.f;
-            float u = v[0];
-#pragma unroll
-            for (int q = 1; q < 8; ++q)
-                if (q < CS)
-                    u += v[q];
-            if (row == 0)
-                u0[t] = u;
-            else
-                uT[t * p.rp + row - 1] = u;
-        }
-        for (int e = tid; e < TOK * (p.rp - p.r); e += kThreads) {
-            const int t = e / (p.rp - p.r), j = p.r + e - t * (p.rp - p.r);
-            uT[t * p.rp + j] = 0.f;
-        }
+    if (!kOverlap && p.JB > 0) {
+        if (tid < kConsumers)
+            fetch_u(tid, kConsumers, s_good != 0);
         __syncthreads();
-        if (tid == 0 && atomicAdd(&p.flags[1], 1u) == (unsigned)(p.NC - 1)) {
-            // every 64-row cluster has read u: reset for the next forward
-            p.flags[1] = 0u;
-            p.flags[0] = 0u;
-        }
+    }
+    if (p.JB > 0 && tid == 0 && atomicAdd(&p.flags[1], 1u) == (unsigned)(p.NC - 1)) {
+        // every 64-row cluster has read u: reset for the next forward
+        p.flags[1] = 0u;
+        p.flags[0] = 0u;
     }
 
-    // ---- epilogue of a 64-row cluster (256 threads: 64 rows x 4 token phases)
-    if (tid < 256) {
+    // ---- epilogue of a 64-row cluster: consumer thread = row (tid mod 64) and
+    // the tokens th + kPh * i, th = tid / 64
+    constexpr int kPh = kConsumers / 64;
+    constexpr int kTokPerThread = TOK / kPh;
+    if (tid < kConsumers) {
         if (p.JB > 0 && !wait_bounded(bar_bt, 0))
             atomicOr(p.status, kStatusTimeout);
         const int row = tid & (kRows - 1), th = tid >> 6;
         const int64_t n = n0 + row;
-        float out[TOK / 4];
+        float out[kTokPerThread];
 #pragma unroll
-        for (int i = 0; i < TOK / 4; ++i)
-            out[i] = s_epi * red[row * TOK + th + 4 * i];
+        for (int i = 0; i < kTokPerThread; ++i)
+            out[i] = s_epi * red[row * TOK + th + kPh * i];
         if (p.JB > 0) {
             // corr = g_t * sum_j u[1 + j][t] * B^T[n][j]: the B^T row in 16-byte pieces,
-            // u broadcast, both from shared memory
-            float corr[TOK / 4];
+            // u from shared memory.  With one token per thread the pieces start at
+            // a row-dependent offset, spreading the rows over the banks; with
+            // several, all lanes take the same piece and u is a broadcast.
+            float corr[kTokPerThread];
 #pragma unroll
-            for (int i = 0; i < TOK / 4; ++i)
+            for (int i = 0; i < kTokPerThread; ++i)
                 corr[i] = 0.f;
             const uint16_t *btrow = reinterpret_cast<const uint16_t *>(bp + L.bt) + row * p.rp;
-            for (int j0 = 0; j0 < p.rp; j0 += 8) {
+            const int npiece = p.rp / 8;
+            int piece = kTokPerThread == 1 ? (row & (npiece - 1)) : 0;   // start in [0, npiece)
+            for (int pc = 0; pc < npiece; ++pc) {
+                const int j0 = 8 * piece;
+                if (++piece == npiece)
+                    piece = 0;
                 const uint4 bv = *reinterpret_cast<const uint4 *>(btrow + j0);
                 const float bj[8] = {bf16_lo(bv.x), bf16_hi(bv.x), bf16_lo(bv.y), bf16_hi(bv.y),
                                      bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
 #pragma unroll
-                for (int i = 0; i < TOK / 4; ++i) {
-                    const float4 *ut = reinterpret_cast<const float4 *>(uT + (th + 4 * i) * p.rp + j0);
+                for (int i = 0; i < kTokPerThread; ++i) {
+                    const float4 *ut = reinterpret_cast<const float4 *>(uT + (th + kPh * i) * p.rp + j0);
                     const float4 v0 = ut[0], v1 = ut[1];
                     corr[i] += v0.x * bj[0] + v0.y * bj[1] + v0.z * bj[2] + v0.w * bj[3] + v1.x * bj[4] +
                                v1.y * bj[5] + v1.z * bj[6] + v1.w * bj[7];
                 }
             }
 #pragma unroll
-            for (int i = 0; i < TOK / 4; ++i) {
-                const float g = 1.0f / (1.0f + expf(-(u0[th + 4 * i] + p.b_g)));
+            for (int i = 0; i < kTokPerThread; ++i) {
+                const float g = 1.0f / (1.0f + expf(-(u0[th + kPh * i] + p.b_g)));
                 out[i] += g * corr[i];
             }
         }
 #pragma unroll
-        for (int i = 0; i < TOK / 4; ++i) {
-            const int t = th + 4 * i;
+        for (int i = 0; i < kTokPerThread; ++i) {
+            const int t = th + kPh * i;
             if (t < p.M && n < p.N)
                 p.y[(int64_t)t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
         }
