@@ -108,6 +108,12 @@ def traffic_per_launch(workload, Ms):
     return round(sum(t["bytes"][M] for M in Ms) / len(Ms))
 
 
+def path_name(choice):
+    from w4_gemm_error_b200 import spear
+    path = "decode" if choice & spear.SPEAR_FORCE_DECODE else "tcgen05"
+    return path + ("+split" if choice & spear.SPEAR_FORCE_SPLIT else "+fused")
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -215,6 +221,13 @@ def run_ours(args, rank, world, local_rank):
 
     xs = {M: make_x(M, K, seed=0).to(dev) for M in Ms}
     bufs = {M: [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)] for M in Ms}
+    if not args.no_tune:
+        # the library's adaptive dispatch: each layer times its legal paths once per batch size
+        with torch.cuda.stream(stream):
+            for M in Ms:
+                for lin in layers:
+                    lin.tune(xs[M], bufs[M][0], stream=stream)
+        torch.cuda.synchronize(dev)
 
     def step(flags=0):
         for M in Ms:
@@ -348,6 +361,8 @@ def run_ours(args, rank, world, local_rank):
                        "l2": f"inputs larger than L2: {L} distinct packed layers, "
                              f"{packed_bytes(K, N, r) * L / 1e6:.0f} MB > 3 x 126 MB",
                        "graph": "one CUDA graph per step, kernels chained with programmatic dependent launch",
+                       "dispatch": "untuned" if args.no_tune else "tuned (spear_w4ec_tune per layer and M)",
+                       "paths": {str(M): path_name(layers[0].dispatch(M)) for M in Ms},
                        "parallelism": f"replicas x{world}"},
             "ec_overhead": round(ec_overhead, 4),
             "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d,
@@ -461,6 +476,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=0, help="layers in the stack (0: enough to exceed 3x L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-tune", action="store_true", help="keep the library's untuned dispatch")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
