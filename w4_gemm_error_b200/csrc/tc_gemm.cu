@@ -12,27 +12,30 @@
 //     D[n, t] = sum_k (q[n,k] - z[n]) x[t,k] + sum_j (B[j,n] / s[n]) v[t,j]
 // and the epilogue writes y[t, n] = bf16(s[n] * D[n, t]).
 //
-// Layout of one CTA (persistent, one per SM, 14 warps):
-//   warp 0      TMA producer: x tile (256 tokens x 64 k, 128B-swizzled) and
+// Layout of one CTA (persistent, one per SM, 22 warps):
+//   warp 0      TMA producer: x tile (BN tokens x 64 k, 128B-swizzled) and
 //               the int4 code tile (128 rows x 64 k) per stage; for the EC
 //               stages the B^T/s tile and the v tile (32 fp32 j each) instead.
 //   warp 1      TMEM allocator and the single MMA-issuing thread:
 //               tcgen05.mma.cta_group::1.kind::f16, M = 128 weight rows,
-//               N = 256 tokens, K = 16 per instruction (swap-AB: weights
-//               on the M side so one dequantised tile serves 256 tokens).
-//   warps 2-9   dequantisers: thread (i, h) owns half h of weight row i of
-//               the tile (32 k) and writes the exact integers (q - z) as
-//               bf16 into the 128B-swizzled K-major A tile of the stage (the
-//               layout the MMA descriptor names); two warps per SM sub-
-//               partition so one hides the other's latency.
-//   warps 10-13 epilogue: tcgen05.ld of the finished accumulator (each warp
+//               N = BN tokens (32, 64, 128 or 256: the narrowest that holds
+//               the batch), K = 16 per instruction (swap-AB: weights on the
+//               M side so one dequantised tile serves BN tokens).
+//   warps 2-17  dequantisers, two groups of eight warps taking alternate
+//               stages (a stage's wait, code load, conversion, stores and
+//               fence form a latency chain; two groups keep two stages in
+//               conversion at once): thread (i, h) of a group owns half h of
+//               weight row i of the tile (32 k) and writes the exact integers
+//               (q - z) as bf16 into the 128B-swizzled K-major A tile of the
+//               stage (the layout the MMA descriptor names).
+//   warps 18-21 epilogue: tcgen05.ld of the finished accumulator (each warp
 //               its 32-lane quarter), times the channel scale s[n], bf16
 //               rounding, stores of y[t, n].
 // The accumulator holds sum_k x (q - z) exactly up to fp32 summation, so the
 // EC stages use B^T / s[n] (prepared at pack time) and one multiplication by
 // s[n] in the epilogue scales both terms.
-// Four stages of 52 KB in shared memory; two 256-column accumulators in
-// TMEM so the epilogue of one tile overlaps the main loop of the next.
+// 4 to 8 stages (about 200 KB) in shared memory; two BN-column accumulators
+// in TMEM so the epilogue of one tile overlaps the main loop of the next.
 // Every mbarrier wait is bounded (about a second of SM clock cycles); a wait
 // that runs out sets the handle's status word and the kernel winds down.
 #include <new>
@@ -45,16 +48,19 @@ namespace spear {
 namespace {
 
 constexpr int BM = 128;                       // weight rows per tile (TMEM lanes)
-constexpr int BN = 256;                       // tokens per tile (MMA N)
 constexpr int BK = 64;                        // k per stage: one 128-byte swizzle atom of bf16
-constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;          // 16 KB dequantised weights (or B^T on EC stages)
-constexpr int B_BYTES = BN * BK * 2;          // 32 KB activations (or v on EC stages)
 constexpr int C_BYTES = BM * BK / 2;          // 4 KB int4 codes
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-constexpr int THREADS = 448;   // 14 warps: TMA, MMA, 8 dequantisers, 4 epilogue
-constexpr int TMEM_COLS = 2 * BN;
+constexpr int THREADS = 704;   // 22 warps: TMA, MMA, 2 x 8 dequantisers, 4 epilogue
+
+// Token tile BN (the MMA N: 32, 64, 128 or 256) and what depends on it: the
+// activation tile of a stage (BN x 64 bf16, or v on EC stages), the ring depth
+// (more stages for narrower tiles, within about 210 KB) and two accumulators of
+// BN columns in TMEM.
+__host__ __device__ constexpr int tc_b_bytes(int BN) { return BN * BK * 2; }
+__host__ __device__ constexpr int tc_stage_bytes(int BN) { return A_BYTES + tc_b_bytes(BN) + C_BYTES; }
+__host__ __device__ constexpr int tc_stages(int BN) { return BN >= 256 ? 4 : (BN >= 128 ? 6 : (BN >= 64 ? 7 : 8)); }
+__host__ __device__ constexpr int tc_smem_bytes(int BN) { return tc_stages(BN) * tc_stage_bytes(BN) + 1024; }
 
 struct TcParams {
     int64_t M, N;
@@ -223,10 +229,15 @@ tc_prepass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
 
 // ---------------------------------------------------------------- the kernel
 
+template <int BN>
 __global__ void __launch_bounds__(THREADS, 1)
 tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
                const __grid_constant__ CUtensorMap tm_bt, const __grid_constant__ CUtensorMap tm_v, TcParams p)
 {
+    constexpr int STAGES = tc_stages(BN);
+    constexpr int B_BYTES = tc_b_bytes(BN);
+    constexpr int STAGE_BYTES = tc_stage_bytes(BN);
+    constexpr int TMEM_COLS = 2 * BN;
     extern __shared__ uint8_t smem_raw[];
     __shared__ __align__(8) uint64_t bars[3 * STAGES + 5];
     __shared__ uint32_t tmem_base_slot;
@@ -356,9 +367,12 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             mma_commit(drain);
             mbar_wait_final(drain, 0);
         }
-    } else if (warp < 10) {
-        // ------------------------------------------------ dequantisers: thread (i, h) = half h of weight row i
-        const int i = (tid - 64) & 127, half = (tid - 64) >> 7;
+    } else if (warp < 18) {
+        // ------------------------------------------------ dequantisers: group `grp` takes the stages
+        // g with g % 2 == grp; its thread (i, h) = half h of weight row i
+        const int dq = tid - 64;
+        const uint32_t grp = (uint32_t)(dq >> 8);
+        const int i = dq & 127, half = (dq >> 7) & 1;
         uint32_t g = 0;
         for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
             const int n = (tile / p.n_ttiles) * BM + i;
@@ -366,6 +380,8 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const uint32_t negz = zb | (zb << 16);
             bool ok = true;
             for (int st = 0; st < n_stages; ++st, ++g) {
+                if ((g & 1u) != grp)
+                    continue;
                 const uint32_t slot = g % STAGES, phase = (g / STAGES) & 1;
                 if (!mbar_wait(full0 + 8 * slot, phase, &abort_flag, p.status)) {
                     ok = false;
@@ -488,14 +504,17 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
         const int bits = kStatusTimeout;
         return cudaMemcpyAsync(status, &bits, sizeof(int), cudaMemcpyHostToDevice, st);
     }
+    // token tile: the narrowest of 32, 64, 128, 256 that holds M (one tile row of tokens
+    // up to 256), so that small batches do not run 256-wide MMAs on zero rows
+    const int BN = M <= 32 ? 32 : (M <= 64 ? 64 : (M <= 128 ? 128 : 256));
     CUtensorMap tm_x, tm_v;
-    cudaError_t e = make_map(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.K, (uint64_t)M, BK, BN,
-                             CU_TENSOR_MAP_SWIZZLE_128B);
+    cudaError_t e = make_map(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.K, (uint64_t)M, BK,
+                             (uint32_t)BN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess)
         return e;
     const bool use_ec = ec && pk.r > 0;
     if (use_ec) {
-        e = make_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)pk.rp, (uint64_t)M, 32, BN,
+        e = make_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)pk.rp, (uint64_t)M, 32, (uint32_t)BN,
                      CU_TENSOR_MAP_SWIZZLE_128B);
         if (e != cudaSuccess)
             return e;
@@ -516,20 +535,31 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
     p.y = static_cast<uint16_t *>(y);
     p.status = status;
 
-    e = raise_smem_limit(reinterpret_cast<const void *>(tc_w4ec_kernel), SMEM_BYTES);
+    const void *fn = BN == 32 ? reinterpret_cast<const void *>(tc_w4ec_kernel<32>)
+                   : BN == 64 ? reinterpret_cast<const void *>(tc_w4ec_kernel<64>)
+                   : BN == 128 ? reinterpret_cast<const void *>(tc_w4ec_kernel<128>)
+                               : reinterpret_cast<const void *>(tc_w4ec_kernel<256>);
+    const int smem = tc_smem_bytes(BN);
+    e = raise_smem_limit(fn, smem);
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(p.n_tiles < num_sms ? p.n_tiles : num_sms));
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, tc_w4ec_kernel, tm_x, m->codes, use_ec ? m->bt : m->codes, tm_v, p);
+    const CUtensorMap &bt = use_ec ? m->bt : m->codes;
+    switch (BN) {
+    case 32: return cudaLaunchKernelEx(&cfg, tc_w4ec_kernel<32>, tm_x, m->codes, bt, tm_v, p);
+    case 64: return cudaLaunchKernelEx(&cfg, tc_w4ec_kernel<64>, tm_x, m->codes, bt, tm_v, p);
+    case 128: return cudaLaunchKernelEx(&cfg, tc_w4ec_kernel<128>, tm_x, m->codes, bt, tm_v, p);
+    default: return cudaLaunchKernelEx(&cfg, tc_w4ec_kernel<256>, tm_x, m->codes, bt, tm_v, p);
+    }
 }
 
 }  // namespace spear
