@@ -111,7 +111,6 @@ tc_prepass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
 
-    pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
     const uint32_t x_bytes = 128 * 128, g_bytes = (uint32_t)p.R1p * 128;
@@ -144,6 +143,10 @@ tc_prepass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_slot;
+    // let the next kernel start only now that this CTA holds its tensor memory:
+    // a dependent CTA that cannot allocate then waits for a kernel that needs
+    // nothing from it
+    pdl_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -243,7 +246,6 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
 
-    pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
     uint8_t *const base_ptr = smem_raw + (base - smem_addr(smem_raw));
@@ -279,6 +281,9 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_slot;
+    // let the next kernel start only now that this CTA holds its tensor memory
+    // (see the prepass kernel)
+    pdl_launch_dependents();
     const int n_stages = p.n_main + p.n_ec;
 
     if (warp == 0) {
