@@ -82,13 +82,13 @@ def packed_bytes(K, N, r):
 TRAFFIC = {
     "decode_qo_4096x4096_r32": dict(
         kernel="decode_w4ec_kernel",
-        files=("decode.cu", "async_utils.cuh", "device_utils.cuh", "kernels.h"), sha="9dae823ec82d3bfe",
-        bytes={1: 9.1407e6, 4: 9.1618e6, 16: 9.2533e6},
+        files=("decode.cu", "async_utils.cuh", "device_utils.cuh", "kernels.h"), sha="6f817795c9c902f2",
+        bytes={1: 9.1372e6, 4: 9.1631e6, 16: 9.2537e6},
         profile="profiles/decode_w4ec_kernel_decode_qo_4096x4096_r32.md"),
     "prefill_mlp_4096x14336_r64": dict(
         kernel="tc_w4ec_kernel",
-        files=("tc_gemm.cu", "tc_gemm.h", "async_utils.cuh", "device_utils.cuh"), sha="6979bcf5ac40d881",
-        bytes={2048: 69.365e6, 4096: 156.326e6},
+        files=("tc_gemm.cu", "tc_gemm.h", "async_utils.cuh", "device_utils.cuh"), sha="2cffdf5564c5e6af",
+        bytes={2048: 69.387e6, 4096: 156.332e6},
         profile="profiles/tc_w4ec_kernel_prefill_mlp_4096x14336_r64.md"),
 }
 

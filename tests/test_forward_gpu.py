@@ -224,9 +224,11 @@ def test_injected_faults_are_reported(monkeypatch):
 
 # ------------------------------------------------------------------ tcgen05 tile kernel
 
+# token tiles of 32 (M <= 32), 64, 128 and 256 columns
 @pytest.mark.parametrize("M,K,N,r", [(33, 256, 128, 8), (256, 4096, 1024, 64), (300, 512, 256, 32),
                                      (1000, 1032, 264, 20), (513, 4104, 136, 33), (64, 2048, 512, 32),
-                                     (9, 8, 8, 1), (700, 8192, 256, 128)])
+                                     (9, 8, 8, 1), (700, 8192, 256, 128), (100, 1032, 264, 20),
+                                     (128, 512, 384, 16), (32, 4096, 256, 64)])
 def test_tc_path_shapes(M, K, N, r):
     P = Problem(M, K, N, r, seed=M + N)
     ref = P.oracle_y()
