@@ -137,9 +137,8 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
 /* The flags (path | fused/split) that forward would use for M tokens now:
  * the tuned choice of M's bucket if spear_w4ec_tune has filled it, else the
  * default rule (fused EC; the decode kernel up to 32 tokens; beyond, the
- * tcgen05 kernel, unless its 128-row x 256-token tiles would occupy fewer than
- * half of the SMs for up to 128 tokens, where the decode kernel runs 32-token
- * slices). */
+ * tcgen05 kernel, which splits K for up to 128 tokens on layers whose 128-row
+ * tiles fill at most half of the SMs). */
 int spear_w4ec_dispatch(const spear_w4ec *h, int64_t M, uint32_t *choice);
 
 /* Per-token gate with no allocation at all, for callers that may not call

@@ -127,12 +127,28 @@ __global__ void __launch_bounds__(128) prepass_kernel(PrepassParams p)
             return;
         __threadfence();
         const float *all = p.part + (size_t)tile * p.S * tile_elems;
-        for (int e = tid; e < tile_elems; e += 128) {
-            float sum = 0.f;
-            for (int q = 0; q < p.S; ++q)
-                sum += __ldcg(all + (size_t)q * tile_elems + e);
-            red[e] = sum;
+        // thread tid sums the elements tid + 128 i (i < 2 MT: the tile is 16 MT x 16)
+        // in split order, loading four partials of all of them per round
+        float sum[2 * MT];
+#pragma unroll
+        for (int i = 0; i < 2 * MT; ++i)
+            sum[i] = 0.f;
+        for (int q0 = 0; q0 < p.S; q0 += 4) {
+            float w[4][2 * MT];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int i = 0; i < 2 * MT; ++i)
+                    w[q][i] = q0 + q < p.S ? __ldcg(all + (size_t)(q0 + q) * tile_elems + tid + 128 * i) : 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int i = 0; i < 2 * MT; ++i)
+                    sum[i] += w[q][i];
         }
+#pragma unroll
+        for (int i = 0; i < 2 * MT; ++i)
+            red[tid + 128 * i] = sum[i];
         if (tid == 0)
             p.counters[tile] = 0u;
         __syncthreads();
@@ -163,7 +179,7 @@ int pick_splits(int64_t M, int64_t Kp, int num_sms)
     const int nkb = (int)(Kp / 64);
     int S = std::max(1, (2 * num_sms) / std::max(tiles, 1));
     S = std::min(S, std::max(1, nkb / 4));  // at least one k block per warp
-    return std::min(S, 64);
+    return std::min(S, 32);                  // the last CTA sums them four at a time
 }
 
 using PrepassFn = void (*)(PrepassParams);

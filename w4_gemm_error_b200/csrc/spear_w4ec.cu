@@ -134,16 +134,12 @@ bool tc_supported(const spear_w4ec *h) { return tc_available(h->pk); }
 // table entry, or the default (the split-K decode kernel for a few tokens,
 // the tcgen05 tile kernel above, the EC fused in both).
 // Untuned path: the decode kernel up to 32 tokens; beyond, the tcgen05
-// kernel, unless its 128-row x 256-token output tiles would occupy fewer than
-// half of the SMs for up to 128 tokens (narrow layers with a long K, e.g.
-// 14336 -> 4096), where 32-token decode slices stream the weights faster.
+// kernel (which splits K on layers whose 128-row tiles fill at most half of
+// the SMs).
 uint32_t default_path(const spear_w4ec *h, int64_t M)
 {
     const bool dec = decode_supported(h->pk, h->num_sms);
     if (!tc_supported(h) || (dec && M <= kDecodeMaxTokens))
-        return SPEAR_FORCE_DECODE;
-    const int64_t tiles = (h->pk.Np / 128) * ((M + 255) / 256);
-    if (dec && M <= 128 && 2 * tiles < h->num_sms)
         return SPEAR_FORCE_DECODE;
     return SPEAR_FORCE_TC;
 }

@@ -38,6 +38,7 @@
 // in TMEM so the epilogue of one tile overlaps the main loop of the next.
 // Every mbarrier wait is bounded (about a second of SM clock cycles); a wait
 // that runs out sets the handle's status word and the kernel winds down.
+#include <algorithm>
 #include <new>
 
 #include "async_utils.cuh"
@@ -67,6 +68,12 @@ struct TcParams {
     int kchunks;       // Kp / 256: tiled code blocks per 64-row block
     int n_main, n_ec, rp;
     int n_ttiles, n_tiles;
+    // split K: work unit u = tile * ksplit + ks runs main stages [ks * sps, min((ks + 1) * sps, n_main)),
+    // the last split also the EC stages; with ksplit > 1 each unit writes an fp32 partial tile and the
+    // last unit of a tile to finish sums them in split order
+    int ksplit, sps, n_units;
+    float *part;           // [n_tiles][ksplit][BN][128] fp32
+    unsigned *counters;    // [n_tiles] finished units of each tile
     const float *s;
     const uint8_t *z;
     uint16_t *y;
@@ -245,6 +252,7 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     __shared__ __align__(8) uint64_t bars[3 * STAGES + 5];
     __shared__ uint32_t tmem_base_slot;
     __shared__ volatile int abort_flag;
+    __shared__ volatile int s_last;   // split K: this unit finished its tile
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
@@ -284,7 +292,6 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     // let the next kernel start only now that this CTA holds its tensor memory
     // (see the prepass kernel)
     pdl_launch_dependents();
-    const int n_stages = p.n_main + p.n_ec;
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
@@ -292,9 +299,13 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             pdl_wait();  // x and v come from earlier kernels in the stream
             uint32_t g = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+                const int tile = u / p.ksplit, ks = u - tile * p.ksplit;
                 const int t0 = (tile % p.n_ttiles) * BN, n0 = (tile / p.n_ttiles) * BM;
-                for (int st = 0; st < n_stages; ++st, ++g) {
+                const int lo = ks * p.sps, nm = min(lo + p.sps, p.n_main) - lo;
+                const int nst = nm + (ks == p.ksplit - 1 ? p.n_ec : 0);
+                for (int i = 0; i < nst; ++i, ++g) {
+                    const int st = i < nm ? lo + i : p.n_main + (i - nm);
                     const uint32_t slot = g % STAGES, phase = (g / STAGES) & 1;
                     if (!mbar_wait(empty0 + 8 * slot, phase ^ 1, &abort_flag, p.status)) {
                         ok = false;
@@ -337,13 +348,17 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             uint32_t g = 0;
             int lt = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++lt) {
+            for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x, ++lt) {
                 const uint32_t buf = lt & 1;
                 if (!mbar_wait(tempty0 + 8 * buf, ((lt >> 1) & 1) ^ 1, &abort_flag, p.status))
                     break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + buf * BN;
-                for (int st = 0; st < n_stages; ++st, ++g) {
+                const int ks = u % p.ksplit;
+                const int lo = ks * p.sps, nm = min(lo + p.sps, p.n_main) - lo;
+                const int nst = nm + (ks == p.ksplit - 1 ? p.n_ec : 0);
+                for (int i = 0; i < nst; ++i, ++g) {
+                    const int st = i < nm ? lo + i : p.n_main + (i - nm);
                     const uint32_t slot = g % STAGES, phase = (g / STAGES) & 1;
                     if (!mbar_wait(full0 + 8 * slot, phase, &abort_flag, p.status) ||
                         !mbar_wait(aready0 + 8 * slot, phase, &abort_flag, p.status)) {
@@ -355,7 +370,7 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     const uint64_t a_desc = smem_desc_sw128(sb), b_desc = smem_desc_sw128(sb + A_BYTES);
                     if (st < p.n_main) {
                         for (int k = 0; k < BK / 16; ++k)
-                            mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (st > 0 || k > 0) ? 1u : 0u);
+                            mma_bf16(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, (i > 0 || k > 0) ? 1u : 0u);
                     } else {
                         // EC: 32 tf32 values of j per 128-byte row, 8 per instruction
                         const int rem = p.rp - (st - p.n_main) * 32;
@@ -379,14 +394,18 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const uint32_t grp = (uint32_t)(dq >> 8);
         const int i = dq & 127, half = (dq >> 7) & 1;
         uint32_t g = 0;
-        for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
+        for (int u = blockIdx.x; u < p.n_units; u += gridDim.x) {
+            const int tile = u / p.ksplit, ks = u - tile * p.ksplit;
+            const int lo = ks * p.sps, nm = min(lo + p.sps, p.n_main) - lo;
+            const int nst = nm + (ks == p.ksplit - 1 ? p.n_ec : 0);
             const int n = (tile / p.n_ttiles) * BM + i;
             const uint32_t zb = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + p.z[n])));
             const uint32_t negz = zb | (zb << 16);
             bool ok = true;
-            for (int st = 0; st < n_stages; ++st, ++g) {
+            for (int ii = 0; ii < nst; ++ii, ++g) {
                 if ((g & 1u) != grp)
                     continue;
+                const int st = ii < nm ? lo + ii : p.n_main + (ii - nm);
                 const uint32_t slot = g % STAGES, phase = (g / STAGES) & 1;
                 if (!mbar_wait(full0 + 8 * slot, phase, &abort_flag, p.status)) {
                     ok = false;
@@ -423,7 +442,8 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         const int q = warp & 3;
         const int row = 32 * q + lane;
         int lt = 0;
-        for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++lt) {
+        for (int u = blockIdx.x; u < p.n_units; u += gridDim.x, ++lt) {
+            const int tile = u / p.ksplit, ks = u - tile * p.ksplit;
             const uint32_t buf = lt & 1;
             if (!mbar_wait(tfull0 + 8 * buf, (lt >> 1) & 1, &abort_flag, p.status))
                 break;
@@ -432,21 +452,73 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const int64_t n = (int64_t)(tile / p.n_ttiles) * BM + row;
             const float sn = p.s[n];
             const float e_n = sn != 0.0f ? sn : 1.0f;   // the EC operand was divided by it
+            if (p.ksplit == 1) {
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
-                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * BN + 32 * c, r);
-                if (n < p.N) {
+                for (int c = 0; c < BN / 32; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * BN + 32 * c, r);
+                    if (n < p.N) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int64_t t = t0 + 32 * c + j;
-                        if (t < p.M)
-                            p.y[t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(e_n * __uint_as_float(r[j])));
+                        for (int j = 0; j < 32; ++j) {
+                            const int64_t t = t0 + 32 * c + j;
+                            if (t < p.M)
+                                p.y[t * p.N + n] =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(e_n * __uint_as_float(r[j])));
+                        }
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(tempty0 + 8 * buf);
+                continue;
+            }
+            // ---- split K: this unit's fp32 partial, token-major so that the 128 rows of
+            // a token are contiguous; the last unit of the tile to finish sums the
+            // partials in split order
+            float *tp = p.part + (size_t)tile * p.ksplit * BN * BM;   // [ksplit][BN][128]
+            const int jn = (int)min((int64_t)BN, p.M - t0);             // tokens of the tile
+#pragma unroll 1
+            for (int c = 0; c < BN / 32 && 32 * c < jn; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(32 * q) << 16) + buf * BN + 32 * c, r);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (32 * c + j < jn)
+                        tp[((size_t)ks * BN + 32 * c + j) * BM + row] = __uint_as_float(r[j]);
             }
             tc_fence_before();
             mbar_arrive(tempty0 + 8 * buf);
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // the four epilogue warps
+            if (q == 0 && lane == 0)
+                s_last = atomicAdd(&p.counters[tile], 1u) == (unsigned)(p.ksplit - 1) ? 1 : 0;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (s_last) {
+                __threadfence();
+                // eight tokens at a time, so that eight loads per part are in flight
+#pragma unroll 1
+                for (int j0 = 0; j0 < jn; j0 += 8) {
+                    float v[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        v[jj] = 0.f;
+                    for (int k2 = 0; k2 < p.ksplit; ++k2) {
+                        float w[8];
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj)
+                            w[jj] = j0 + jj < jn ? __ldcg(tp + ((size_t)k2 * BN + j0 + jj) * BM + row) : 0.f;
+#pragma unroll
+                        for (int jj = 0; jj < 8; ++jj)
+                            v[jj] += w[jj];
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        if (j0 + jj < jn && n < p.N)
+                            p.y[(t0 + j0 + jj) * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(e_n * v[jj]));
+                }
+                if (q == 0 && lane == 0)
+                    p.counters[tile] = 0u;   // for the next forward
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");   // s_last is read before it is rewritten
         }
     }
 
@@ -463,16 +535,46 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
 
 bool tc_available(const Packed &) { return tensor_maps_available(); }
 
-cudaError_t tc_alloc(const Packed &, int64_t, int, TcWork &w)
+// Split K for narrow layers: up to 128 tokens, when the 128-row tiles fill at
+// most half of the SMs, K is split into as many parts as keep one unit per SM
+// (at most 8).  The workspace holds the fp32 partials of every tile at 128
+// tokens (part_floats) and one counter per tile.
+static int max_ksplit(const Packed &pk, int num_sms)
+{
+    const int tiles = (int)(pk.Np / BM);
+    if (2 * tiles > num_sms)
+        return 1;
+    return std::min(8, num_sms / tiles);
+}
+
+cudaError_t tc_alloc(const Packed &pk, int64_t, int num_sms, TcWork &w)
 {
     w.maps = new (std::nothrow) Maps();
-    return w.maps ? cudaSuccess : cudaErrorMemoryAllocation;
+    if (!w.maps)
+        return cudaErrorMemoryAllocation;
+    const int ks = max_ksplit(pk, num_sms);
+    if (ks < 2)
+        return cudaSuccess;
+    w.n_counters = (int)(pk.Np / BM);
+    w.part_floats = (size_t)ks * (size_t)pk.Np * 128;
+    cudaError_t e = cudaMalloc(&w.part, w.part_floats * sizeof(float));
+    if (e == cudaSuccess)
+        e = cudaMalloc(&w.counters, (size_t)w.n_counters * sizeof(unsigned));
+    if (e == cudaSuccess)
+        e = cudaMemset(w.counters, 0, (size_t)w.n_counters * sizeof(unsigned));
+    return e;
 }
 
 void tc_free(TcWork &w)
 {
     delete static_cast<Maps *>(w.maps);
     w.maps = nullptr;
+    cudaFree(w.part);
+    cudaFree(w.counters);
+    w.part = nullptr;
+    w.counters = nullptr;
+    w.part_floats = 0;
+    w.n_counters = 0;
 }
 
 cudaError_t tc_prepare(const Packed &pk, TcWork &w)
@@ -535,6 +637,15 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
     p.rp = pk.rp;
     p.n_ttiles = (int)((M + BN - 1) / BN);
     p.n_tiles = p.n_ttiles * (int)(pk.Np / BM);
+    // split K (see max_ksplit) with at least 8 stages per part
+    int ks = 1;
+    if (w.part && M <= 128 && p.n_tiles == w.n_counters)
+        ks = std::max(1, std::min(max_ksplit(pk, num_sms), p.n_main / 8));
+    p.sps = (p.n_main + ks - 1) / ks;
+    p.ksplit = (p.n_main + p.sps - 1) / p.sps;   // no empty part
+    p.n_units = p.n_tiles * p.ksplit;
+    p.part = w.part;
+    p.counters = w.counters;
     p.s = pk.s;
     p.z = pk.z;
     p.y = static_cast<uint16_t *>(y);
@@ -549,7 +660,7 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
     if (e != cudaSuccess)
         return e;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(p.n_tiles < num_sms ? p.n_tiles : num_sms));
+    cfg.gridDim = dim3((unsigned)(p.n_units < num_sms ? p.n_units : num_sms));
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
