@@ -251,6 +251,23 @@ def test_tc_path_invariants():
     P.close()
 
 
+def test_tc_split_k_invariants():
+    # a narrow layer (4 row tiles) at 64 tokens: K split four ways, partials summed
+    # by the last unit of each tile in split order, so runs are bit-identical
+    P = Problem(64, 2048, 512, 32, seed=15)
+    y1 = _run(P, TC)
+    for _ in range(3):
+        assert torch.equal(_run(P, TC), y1), "repeated split-K runs differ"
+    y_off = _run(P, TC | EC_OFF)
+    y2 = _run(P, TC | EC_OFF, x=(P.xd.float() * 2).to(torch.bfloat16))
+    assert torch.equal(y2, (y_off.float() * 2).to(torch.bfloat16)), "y(2x) != 2 y(x)"
+    perm = torch.randperm(64, generator=torch.Generator().manual_seed(2))
+    yp = _run(P, TC, x=P.xd[perm.cuda()].contiguous())
+    assert torch.equal(yp, y1[perm.cuda()]), "token permutation"
+    assert_close(y1, P.oracle_y(), "split-K vs oracle")
+    P.close()
+
+
 def test_tc_ec_isolated():
     P = Problem(256, 4096, 1024, 64, seed=14)
     y_on = _run(P, TC).double().cpu().numpy()
