@@ -66,8 +66,9 @@ constexpr int kSmemPerCta = 110 * 1024;
 
 struct Maps {
     CUtensorMap codes;    // tiled codes, one box = one 8 KB block (64 rows x 256 k), 128B swizzle
-    CUtensorMap g;        // [R1p][Kp] bf16, boxes of 64 x 16, 128B swizzle
+    CUtensorMap g;        // [R1p][Kp] bf16 seen as [Kp/64][R1p][64]: one box = 4 x (16 rows x 64 k)
     CUtensorMap bt;       // [Np][rp] bf16, boxes of rp x 64
+    int g3;               // g is the 3-D view (else 2-D boxes of 64 k x 16 rows)
 };
 
 struct DecodeParams {
@@ -84,6 +85,7 @@ struct DecodeParams {
     int JB, NC;           // EC clusters, 64-row clusters
     int r, rp, R1p;
     int push;             // partial tiles pushed into receive slots of the first CTA
+    int x3, g3;           // activations / G rows as one 3-D box per stage (else four 2-D boxes)
     float b_g;
 };
 
@@ -189,8 +191,11 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         const uint32_t bar = bar_full_w + 8 * st;
         mbar_expect_tx(bar, 8192);
         if (is_u) {
-            for (int i = 0; i < 4; ++i)
-                tma_load_2d(dst + i * 2048, &tm_g, k0 + c * kChunk + i * 64, 16 * cluster, bar);
+            if (p.g3)
+                tma_load_3d(dst, &tm_g, 0, 16 * cluster, (k0 + c * kChunk) / 64, bar);
+            else
+                for (int i = 0; i < 4; ++i)
+                    tma_load_2d(dst + i * 2048, &tm_g, k0 + c * kChunk + i * 64, 16 * cluster, bar);
         } else {
             tma_load_3d(dst, &tm_codes, 0, 0, (n0 / kRows) * (int)(p.Kp / kChunk) + (k0 / kChunk) + c, bar);
         }
@@ -199,8 +204,11 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         const uint32_t dst = base + L.ring + st * kStage + 8192;
         const uint32_t bar = bar_full_x + 8 * st;
         mbar_expect_tx(bar, kXBytes);
-        for (int i = 0; i < 4; ++i)
-            tma_load_2d(dst + i * (TOK * 128), &tm_x, k0 + c * kChunk + 64 * i, 0, bar);
+        if (p.x3)
+            tma_load_3d(dst, &tm_x, 0, 0, (k0 + c * kChunk) / 64, bar);
+        else
+            for (int i = 0; i < 4; ++i)
+                tma_load_2d(dst + i * (TOK * 128), &tm_x, k0 + c * kChunk + 64 * i, 0, bar);
     };
 
     if (producer && lane == 0) {
@@ -722,9 +730,21 @@ cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
     cudaError_t e = make_map_nd(&m->codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, dims, strides, box,
                                 CU_TENSOR_MAP_SWIZZLE_128B);
 
-    if (e == cudaSuccess && pk.r > 0)
-        e = make_map(&m->g, pk.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.Kp, (uint64_t)pk.R1p, 64, 16,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
+    m->g3 = 0;
+    if (e == cudaSuccess && pk.r > 0) {
+        // one stage of G rows (16 rows x 256 k) as one box: [k block][row][64 k], laid
+        // out in shared memory as four 2 KB sub-tiles; the 2-D boxes if the driver
+        // does not take this view
+        const uint64_t gd[3] = {64, (uint64_t)pk.R1p, (uint64_t)(pk.Kp / 64)};
+        const uint64_t gs[2] = {(uint64_t)pk.Kp * 2, 128};
+        const uint32_t gb[3] = {64, 16, 4};
+        if (make_map_nd(&m->g, pk.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, gd, gs, gb, CU_TENSOR_MAP_SWIZZLE_128B) ==
+            cudaSuccess)
+            m->g3 = 1;
+        else
+            e = make_map(&m->g, pk.G, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.Kp, (uint64_t)pk.R1p, 64, 16,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+    }
     if (e == cudaSuccess && pk.r > 0)
         e = make_map(&m->bt, pk.Bt, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.rp, (uint64_t)pk.Np,
                      (uint32_t)pk.rp, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
@@ -778,11 +798,25 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     p.R1p = use_ec ? pk.R1p : 0;
     p.b_g = pk.b_g;
     const int T = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
+    // the activations of one stage (TOK rows x 256 k) as one box of the view
+    // [k block][token][64 k] when K is a multiple of 64 (then no box reads past
+    // the end of a row), else as four 2-D boxes with k >= K filled with zeros
     CUtensorMap tm_x;
-    cudaError_t e = make_map(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.K, (uint64_t)M, 64,
-                             (uint32_t)(8 * T), CU_TENSOR_MAP_SWIZZLE_128B);
+    cudaError_t e = cudaErrorInvalidValue;
+    p.x3 = 0;
+    if (pk.K % 64 == 0) {
+        const uint64_t xd[3] = {64, (uint64_t)M, (uint64_t)(pk.K / 64)};
+        const uint64_t xs[2] = {(uint64_t)pk.K * 2, 128};
+        const uint32_t xb[3] = {64, (uint32_t)(8 * T), 4};
+        e = make_map_nd(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, xd, xs, xb, CU_TENSOR_MAP_SWIZZLE_128B);
+        p.x3 = e == cudaSuccess ? 1 : 0;
+    }
+    if (e != cudaSuccess)
+        e = make_map(&tm_x, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)pk.K, (uint64_t)M, 64,
+                     (uint32_t)(8 * T), CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess)
         return e;
+    p.g3 = m->g3;
     const int W = pick_warps(T, p.nch);
     const Plan pl = T == 1 ? plan_for<8>(p.nch, p.rp, CS, W)
                            : (T == 2 ? plan_for<16>(p.nch, p.rp, CS, W) : plan_for<32>(p.nch, p.rp, CS, W));
