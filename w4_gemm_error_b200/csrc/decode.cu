@@ -69,6 +69,7 @@ struct Maps {
     CUtensorMap g;        // [R1p][Kp] bf16 seen as [Kp/64][R1p][64]: one box = 4 x (16 rows x 64 k)
     CUtensorMap bt;       // [Np][rp] bf16, boxes of rp x 64
     int g3;               // g is the 3-D view (else 2-D boxes of 64 k x 16 rows)
+    void *rows;           // maps of the row-CTA kernel (decode_rows.cu), null if it does not fit
 };
 
 struct DecodeParams {
@@ -753,11 +754,15 @@ cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
         m->g = m->codes;
         m->bt = m->codes;
     }
+    if (e == cudaSuccess && decode_rows_shape(pk))
+        e = decode_rows_prepare(pk, &m->rows);
     return e;
 }
 
 void decode_free(DecodeWork &w)
 {
+    if (w.maps)
+        decode_rows_free(static_cast<Maps *>(w.maps)->rows);
     delete static_cast<Maps *>(w.maps);
     w.maps = nullptr;
 }
@@ -773,6 +778,10 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     if (M > kDecodeMaxTokens || !w.maps)
         return cudaErrorInvalidValue;
     const Maps *m = static_cast<const Maps *>(w.maps);
+    // up to 16 tokens on a layer whose 16-row slices fit in shared memory: one
+    // CTA per 16 rows over the whole of K, no exchange between CTAs
+    if (m->rows && decode_rows_fits(pk, M, num_sms))
+        return launch_decode_rows(pk, m->rows, x, y, M, ec, w.ws_u, w.flags, status, st, num_sms);
     const bool use_ec = ec && pk.r > 0;
     DecodeParams p;
     p.Bt = pk.Bt;

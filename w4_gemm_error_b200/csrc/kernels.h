@@ -77,6 +77,17 @@ size_t decode_u_floats(const Packed &pk);
 cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, bool ec, const DecodeWork &w,
                           int *status, cudaStream_t st, int num_sms);
 
+// ---- decode kernel with one CTA per 16 weight rows over the whole of K (up to
+// 16 tokens, K a multiple of 64 and at most 8192, a grid of one wave of two
+// CTAs per SM); launch_decode takes it when it fits.  `maps` is filled by
+// decode_rows_prepare; ws_u and flags are the DecodeWork buffers.
+bool decode_rows_shape(const Packed &pk);
+bool decode_rows_fits(const Packed &pk, int64_t M, int num_sms);
+cudaError_t decode_rows_prepare(const Packed &pk, void **maps);
+void decode_rows_free(void *maps);
+cudaError_t launch_decode_rows(const Packed &pk, const void *maps, const void *x, void *y, int64_t M, bool ec,
+                               float *ws_u, unsigned *flags, int *status, cudaStream_t st, int num_sms);
+
 // ---- split EC: y[t][n] = bf16(y[t][n] + sum_j v[t][j] * Bt[n][j]), v in fp32
 cudaError_t launch_ec_apply(const Packed &pk, const float *vf, void *y, int64_t M, cudaStream_t st);
 
