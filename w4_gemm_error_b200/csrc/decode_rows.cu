@@ -44,6 +44,7 @@ constexpr int kUStrideR = 32;     // token stride of the published u rows (as th
 constexpr int kMaxBoxes = 4;      // TMA boxes per CTA (K <= 8192)
 constexpr int kRowsMaxK = 8192;
 constexpr int kRowsMaxTokens = 16;
+constexpr size_t kRowsSmemPerCta = 112 * 1024;   // two CTAs per SM
 
 struct RowsMaps {
     CUtensorMap codes;   // tiled codes seen as [blocks][64 rows][32 words]: box 32 x 16 rows x cb blocks
@@ -67,6 +68,8 @@ struct RowsParams {
     int JB, NR;           // 16-row groups of G (0 without the EC), row CTAs
     int r, rp, R1p;
     uint32_t region;      // bytes of the codes / G region of shared memory
+    uint32_t xs_off;      // byte offset of the staged activations
+    int xstage;           // the activations are staged in shared memory (a few tokens)
     float b_g;
 };
 
@@ -102,9 +105,9 @@ __host__ __device__ constexpr uint32_t rows_tail_bytes(int W, int rp)
     return (uint32_t)(W * TOK * kRowsPerCta * 4 + 32 * rp + 4 * TOK * (1 + rp));
 }
 
-// Register budget: two CTAs per SM.
-template <int T, int W>
-__global__ void __launch_bounds__(32 * W + 32, 2)
+// Register budget: MINB CTAs per SM.
+template <int T, int W, int MINB>
+__global__ void __launch_bounds__(32 * W + 32, MINB)
 decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_g,
                    RowsParams p)
 {
@@ -175,7 +178,6 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             if (tid < kEpi)
                 s_epi = __ldg(p.s + n0 + (tid & (kRowsPerCta - 1)));
         }
-        const int sb0 = warp * nsb_cta / W, sb1 = (warp + 1) * nsb_cta / W;
         const int64_t kbase = is_u ? (int64_t)qk * nsb_cta * 64 : 0;
         float acc[T][4], acc2[T][4];
 #pragma unroll
@@ -184,27 +186,111 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             for (int i = 0; i < 4; ++i)
                 acc[n][i] = acc2[n][i] = 0.f;
 
-        // activations k = kbase + 64 sb + 16 cl + {0..15} of token 8n + gid (zero
-        // beyond M and K); written by the previous kernel
-        auto load_x = [&](int sb, uint4 (&dst)[T][2]) {
-            const int64_t k = kbase + (int64_t)sb * 64 + 16 * cl;
+        // one 64-k sub-block of the product, activations in xv
+        auto product = [&](int sb, const uint4 (&xv)[T][2]) {
+            if (!is_u) {
+                // codes k = 64 sb + 16 cl + {0..15} of rows gid and gid + 8 (8 bytes
+                // each) in chunk sb / 4, a [16 rows][128 B] tile with the 128B swizzle
+                const uint8_t *ct = bp + (sb >> 2) * 2048;
+                const int unit = ((2 * (sb & 3) + (cl >> 1)) ^ gid) * 16 + (cl & 1) * 8;
+                const uint2 wgv = *reinterpret_cast<const uint2 *>(ct + gid * 128 + unit);
+                const uint2 whv = *reinterpret_cast<const uint2 *>(ct + (gid + 8) * 128 + unit);
 #pragma unroll
-            for (int n = 0; n < T; ++n) {
-                const int64_t t = 8 * n + gid;
-                if (t < p.M && k < p.K) {
-                    const uint16_t *src = p.x + t * p.K + k;
-                    dst[n][0] = ld_nc(src);
-                    dst[n][1] = ld_nc(src + 8);
-                } else {
-                    dst[n][0] = make_uint4(0, 0, 0, 0);
-                    dst[n][1] = dst[n][0];
+                for (int j = 0; j < 2; ++j) {
+                    const uint32_t wgw = j ? wgv.y : wgv.x, whw = j ? whv.y : whv.x;
+                    // codes k = 8j + {0..7}: nibbles (m, m + 4) hold the pair k = 2m, 2m + 1,
+                    // the order of the activations in one uint4
+                    const uint32_t g0 = dequant_pair(wgw, negg), g1 = dequant_pair(wgw >> 4, negg);
+                    const uint32_t g2 = dequant_pair(wgw >> 8, negg), g3 = dequant_pair(wgw >> 12, negg);
+                    const uint32_t h0 = dequant_pair(whw, negh), h1 = dequant_pair(whw >> 4, negh);
+                    const uint32_t h2 = dequant_pair(whw >> 8, negh), h3 = dequant_pair(whw >> 12, negh);
+#pragma unroll
+                    for (int n = 0; n < T; ++n) {
+                        const uint4 v = xv[n][j];
+                        float (&a)[4] = j ? acc2[n] : acc[n];
+                        mma_bf16_16816(a, g0, h0, g1, h1, v.x, v.y);
+                        mma_bf16_16816(a, g2, h2, g3, h3, v.z, v.w);
+                    }
+                }
+            } else {
+                // 16 rows of G, k = 64 sb + 16 cl + {0..15}: natural pairs, step s
+                // covering k = 16 cl + 4s + {0,1} and + {2,3}
+                const uint8_t *gt = bp + sb * 2048;
+                const uint4 a0 = *reinterpret_cast<const uint4 *>(gt + gid * 128 + (((2 * cl) ^ gid) << 4));
+                const uint4 a1 = *reinterpret_cast<const uint4 *>(gt + gid * 128 + (((2 * cl + 1) ^ gid) << 4));
+                const uint4 b0 = *reinterpret_cast<const uint4 *>(gt + (gid + 8) * 128 + (((2 * cl) ^ gid) << 4));
+                const uint4 b1 =
+                    *reinterpret_cast<const uint4 *>(gt + (gid + 8) * 128 + (((2 * cl + 1) ^ gid) << 4));
+                const uint32_t ga[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const uint32_t ha[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int n = 0; n < T; ++n) {
+                    const uint32_t xa[8] = {xv[n][0].x, xv[n][0].y, xv[n][0].z, xv[n][0].w,
+                                            xv[n][1].x, xv[n][1].y, xv[n][1].z, xv[n][1].w};
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        mma_bf16_16816((s & 1) ? acc2[n] : acc[n], ga[2 * s], ha[2 * s], ga[2 * s + 1],
+                                       ha[2 * s + 1], xa[2 * s], xa[2 * s + 1]);
                 }
             }
         };
-
+        const int sb0 = warp * nsb_cta / W, sb1 = (warp + 1) * nsb_cta / W;
         pdl_wait();
         bool ok = true;
-        if (sb0 < sb1) {
+        if (p.xstage) {
+            // A few tokens: the CTA's activations x[t][kbase .. kbase + 64 nsb_cta)
+            // are staged in shared memory first, one round trip for all of them
+            // (rows padded by 16 bytes to spread them over the banks).
+            const int xst = nsb_cta * 64 + 8;
+            uint16_t *const xs = reinterpret_cast<uint16_t *>(bp + p.xs_off);
+            const int mrows = p.M < TOK ? (int)p.M : TOK;
+            const int per_row = nsb_cta * 8;
+            for (int c = tid; c < mrows * per_row; c += kConsumers) {
+                const int t = c / per_row, c8 = c - t * per_row;
+                const int64_t k = kbase + 8 * c8;
+                const uint4 v = k < p.K ? ld_nc(p.x + (int64_t)t * p.K + k) : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(xs + t * xst + 8 * c8) = v;
+            }
+            named_bar_sync(2, kConsumers);
+            if (sb0 < sb1) {
+                for (int b = sb0 / spb; b <= (sb1 - 1) / spb && ok; ++b)
+                    ok = mbar_wait_bounded(smem_addr(&bars[b]), 0);
+                for (int sb = sb0; sb < sb1 && ok; ++sb) {
+                    uint4 xv[T][2];
+#pragma unroll
+                    for (int n = 0; n < T; ++n) {
+                        const int t = 8 * n + gid;
+                        if (t < p.M) {
+                            const uint16_t *src = xs + t * xst + sb * 64 + 16 * cl;
+                            xv[n][0] = *reinterpret_cast<const uint4 *>(src);
+                            xv[n][1] = *reinterpret_cast<const uint4 *>(src + 8);
+                        } else {
+                            xv[n][0] = make_uint4(0, 0, 0, 0);
+                            xv[n][1] = xv[n][0];
+                        }
+                    }
+                    product(sb, xv);
+                }
+            }
+        } else if (sb0 < sb1) {
+            // More tokens: every CTA staging all of x would multiply the traffic
+            // from L2; each warp reads its own activations from global memory,
+            // one sub-block ahead.
+            auto load_x = [&](int sb, uint4 (&dst)[T][2]) {
+                const int64_t k = kbase + (int64_t)sb * 64 + 16 * cl;
+#pragma unroll
+                for (int n = 0; n < T; ++n) {
+                    const int64_t t = 8 * n + gid;
+                    if (t < p.M && k < p.K) {
+                        const uint16_t *src = p.x + t * p.K + k;
+                        dst[n][0] = ld_nc(src);
+                        dst[n][1] = ld_nc(src + 8);
+                    } else {
+                        dst[n][0] = make_uint4(0, 0, 0, 0);
+                        dst[n][1] = dst[n][0];
+                    }
+                }
+            };
             uint4 xv[T][2], xn[T][2];
             load_x(sb0, xv);
             for (int b = sb0 / spb; b <= (sb1 - 1) / spb && ok; ++b)
@@ -212,51 +298,7 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             for (int sb = sb0; sb < sb1 && ok; ++sb) {
                 if (sb + 1 < sb1)
                     load_x(sb + 1, xn);
-                if (!is_u) {
-                    // codes k = 64 sb + 16 cl + {0..15} of rows gid and gid + 8 (8 bytes
-                    // each) in chunk sb / 4, a [16 rows][128 B] tile with the 128B swizzle
-                    const uint8_t *ct = bp + (sb >> 2) * 2048;
-                    const int unit = ((2 * (sb & 3) + (cl >> 1)) ^ gid) * 16 + (cl & 1) * 8;
-                    const uint2 wgv = *reinterpret_cast<const uint2 *>(ct + gid * 128 + unit);
-                    const uint2 whv = *reinterpret_cast<const uint2 *>(ct + (gid + 8) * 128 + unit);
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const uint32_t wgw = j ? wgv.y : wgv.x, whw = j ? whv.y : whv.x;
-                        // codes k = 8j + {0..7}: nibbles (m, m + 4) hold the pair k = 2m, 2m + 1,
-                        // the order of the activations in one uint4
-                        const uint32_t g0 = dequant_pair(wgw, negg), g1 = dequant_pair(wgw >> 4, negg);
-                        const uint32_t g2 = dequant_pair(wgw >> 8, negg), g3 = dequant_pair(wgw >> 12, negg);
-                        const uint32_t h0 = dequant_pair(whw, negh), h1 = dequant_pair(whw >> 4, negh);
-                        const uint32_t h2 = dequant_pair(whw >> 8, negh), h3 = dequant_pair(whw >> 12, negh);
-#pragma unroll
-                        for (int n = 0; n < T; ++n) {
-                            const uint4 v = xv[n][j];
-                            float (&a)[4] = j ? acc2[n] : acc[n];
-                            mma_bf16_16816(a, g0, h0, g1, h1, v.x, v.y);
-                            mma_bf16_16816(a, g2, h2, g3, h3, v.z, v.w);
-                        }
-                    }
-                } else {
-                    // 16 rows of G, k = 64 sb + 16 cl + {0..15}: natural pairs, step s
-                    // covering k = 16 cl + 4s + {0,1} and + {2,3}
-                    const uint8_t *gt = bp + sb * 2048;
-                    const uint4 a0 = *reinterpret_cast<const uint4 *>(gt + gid * 128 + (((2 * cl) ^ gid) << 4));
-                    const uint4 a1 = *reinterpret_cast<const uint4 *>(gt + gid * 128 + (((2 * cl + 1) ^ gid) << 4));
-                    const uint4 b0 = *reinterpret_cast<const uint4 *>(gt + (gid + 8) * 128 + (((2 * cl) ^ gid) << 4));
-                    const uint4 b1 =
-                        *reinterpret_cast<const uint4 *>(gt + (gid + 8) * 128 + (((2 * cl + 1) ^ gid) << 4));
-                    const uint32_t ga[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-                    const uint32_t ha[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-                    for (int n = 0; n < T; ++n) {
-                        const uint32_t xa[8] = {xv[n][0].x, xv[n][0].y, xv[n][0].z, xv[n][0].w,
-                                                xv[n][1].x, xv[n][1].y, xv[n][1].z, xv[n][1].w};
-#pragma unroll
-                        for (int s = 0; s < 4; ++s)
-                            mma_bf16_16816((s & 1) ? acc2[n] : acc[n], ga[2 * s], ha[2 * s], ga[2 * s + 1],
-                                           ha[2 * s + 1], xa[2 * s], xa[2 * s + 1]);
-                    }
-                }
+                product(sb, xv);
                 if (sb + 1 < sb1) {
 #pragma unroll
                     for (int n = 0; n < T; ++n) {
@@ -302,7 +344,9 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                     sum += red[w * TOK * kRowsPerCta + tid];
                 float out = s_epi * sum;
                 if (p.JB > 0) {
-                    named_bar_sync(1, 32 + kEpi);   // u is in shared memory
+                    named_bar_sync(1, 32 + kEpi);   // u is in shared memory (tokens below M)
+                }
+                if (p.JB > 0 && t < p.M) {
                     const uint16_t *btrow = bts + row * p.rp;
                     const float *ut = uT + t * p.rp;
                     float corr = 0.f;
@@ -335,20 +379,46 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             if (lane == 0)
                 good = wait_count(&p.flags[0], (unsigned)(p.JB * kECSplit), p.status) ? 1 : 0;
             good = __shfl_sync(0xffffffffu, good, 0);
-            for (int e = lane; e < (1 + p.r) * TOK; e += 32) {
-                const int row = e / TOK, t = e - row * TOK;
-                float v[kECSplit];
+            // u[row][4 t4 .. 4 t4 + 3] for rows 0..r and the groups of four tokens
+            // that hold the M real ones, the four quarters summed in order.  This
+            // warp shares its SM with the busy consumer warps, so the loop is kept
+            // short: 16-byte loads, two (row, group) pairs 32 apart per lane in flight.
+            const int mt4 = ((p.M < TOK ? (int)p.M : TOK) + 3) / 4;
+            const int npair = (1 + p.r) * mt4;
+            for (int p0 = lane; p0 < npair; p0 += 64) {
+                float4 v[2][kECSplit];
 #pragma unroll
-                for (int q = 0; q < kECSplit; ++q)
-                    v[q] = good ? __ldcg(p.ws_u + ((int64_t)q * p.R1p + row) * kUStrideR + t) : 0.f;
-                float u = v[0];
+                for (int i = 0; i < 2; ++i) {
+                    const int pr = p0 + 32 * i, row = pr / mt4, t4 = pr - row * mt4;
 #pragma unroll
-                for (int q = 1; q < kECSplit; ++q)
-                    u += v[q];
-                if (row == 0)
-                    u0[t] = u;
-                else
-                    uT[t * p.rp + row - 1] = u;
+                    for (int q = 0; q < kECSplit; ++q)
+                        v[i][q] = (good && pr < npair)
+                                      ? __ldcg(reinterpret_cast<const float4 *>(
+                                            p.ws_u + ((int64_t)q * p.R1p + row) * kUStrideR + 4 * t4))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int pr = p0 + 32 * i, row = pr / mt4, t4 = pr - row * mt4;
+                    if (pr >= npair)
+                        continue;
+                    float4 u = v[i][0];
+#pragma unroll
+                    for (int q = 1; q < kECSplit; ++q) {
+                        u.x += v[i][q].x;
+                        u.y += v[i][q].y;
+                        u.z += v[i][q].z;
+                        u.w += v[i][q].w;
+                    }
+                    const float uu[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        if (row == 0)
+                            u0[4 * t4 + c] = uu[c];
+                        else
+                            uT[(4 * t4 + c) * p.rp + row - 1] = uu[c];
+                    }
+                }
             }
             for (int e = lane; e < TOK * (p.rp - p.r); e += 32) {
                 const int t = e / (p.rp - p.r), j = p.r + e - t * (p.rp - p.r);
@@ -364,10 +434,10 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     }
 }
 
-template <int T, int W>
+template <int T, int W, int MINB>
 const void *rows_ptr()
 {
-    return reinterpret_cast<const void *>(decode_rows_kernel<T, W>);
+    return reinterpret_cast<const void *>(decode_rows_kernel<T, W, MINB>);
 }
 
 // Consumer warps per CTA: sixteen for one token group, eight for two.
@@ -379,6 +449,31 @@ uint32_t rows_region(const Packed &pk, int cb, int gkb)
     const int code_bytes = (nch + cb - 1) / cb * cb * 2048;
     const int g_bytes = pk.r > 0 ? (nch + gkb - 1) / gkb * gkb * 2048 : 0;
     return (uint32_t)std::max(code_bytes, g_bytes);
+}
+
+struct RowsPlan {
+    int T, W, cb, gkb, xstage;
+    uint32_t region, xs_off;
+    size_t smem;
+};
+
+// Token groups, warps and shared-memory layout.  Up to 8 tokens the
+// activations of all of K are staged in shared memory when two CTAs still fit
+// on an SM; for more, staging them in every CTA would cost more L2 traffic
+// than it saves in latency.
+void rows_plan(const Packed &pk, int64_t M, RowsPlan &pl)
+{
+    const int nch = (int)(pk.Kp / 256);
+    pl.T = M <= 8 ? 1 : 2;
+    pl.W = rows_warps(pl.T);
+    pl.cb = std::min(8, nch);
+    pl.gkb = std::min(16, nch);
+    pl.region = rows_region(pk, pl.cb, pl.gkb);
+    const size_t tail = pl.T == 1 ? rows_tail_bytes<8>(pl.W, pk.rp) : rows_tail_bytes<16>(pl.W, pk.rp);
+    pl.xs_off = (uint32_t)((pl.region + tail + 15) / 16 * 16);
+    const size_t xs_bytes = (size_t)std::min<int64_t>(M, 8) * (pk.Kp + 8) * 2;
+    pl.xstage = pl.T == 1 && pl.xs_off + xs_bytes + 1024 <= kRowsSmemPerCta ? 1 : 0;
+    pl.smem = pl.xs_off + (pl.xstage ? xs_bytes : 0) + 1024;
 }
 
 }  // namespace
@@ -457,15 +552,20 @@ cudaError_t launch_decode_rows(const Packed &pk, const void *maps, const void *x
     p.r = pk.r;
     p.rp = pk.rp;
     p.R1p = pk.R1p;
-    p.region = rows_region(pk, p.cb, p.gkb);
+    RowsPlan pl;
+    rows_plan(pk, M, pl);
+    if (pl.cb != m->cb || pl.gkb != m->gkb)
+        return cudaErrorInvalidValue;
+    p.region = pl.region;
+    p.xs_off = pl.xs_off;
+    p.xstage = pl.xstage;
     p.b_g = pk.b_g;
     if (p.nbox > kMaxBoxes || p.ngbox > kMaxBoxes)
         return cudaErrorInvalidValue;
-    const int T = M <= 8 ? 1 : 2;
-    const int W = rows_warps(T);
-    const size_t smem = (size_t)p.region + (T == 1 ? rows_tail_bytes<8>(W, pk.rp) : rows_tail_bytes<16>(W, pk.rp)) +
-                        1024;
-    const void *fn = T == 1 ? rows_ptr<1, 16>() : rows_ptr<2, 8>();
+    const int T = pl.T;
+    const int W = pl.W;
+    const size_t smem = pl.smem;
+    const void *fn = T == 1 ? rows_ptr<1, 16, 2>() : rows_ptr<2, 8, 2>();
     cudaError_t e = raise_smem_limit(fn, smem);
     if (e != cudaSuccess)
         return e;
@@ -480,8 +580,8 @@ cudaError_t launch_decode_rows(const Packed &pk, const void *maps, const void *x
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     if (T == 1)
-        return cudaLaunchKernelEx(&cfg, decode_rows_kernel<1, 16>, m->codes, m->g, p);
-    return cudaLaunchKernelEx(&cfg, decode_rows_kernel<2, 8>, m->codes, m->g, p);
+        return cudaLaunchKernelEx(&cfg, decode_rows_kernel<1, 16, 2>, m->codes, m->g, p);
+    return cudaLaunchKernelEx(&cfg, decode_rows_kernel<2, 8, 2>, m->codes, m->g, p);
 }
 
 }  // namespace spear
