@@ -217,6 +217,11 @@ def run_ours(args, rank, world, local_rank):
             B = torch.roll(B0, shifts=31 * i, dims=1).contiguous()
             layers.append(spear.W4ECLinear(W, A, B, wg, base.b_g, max_M=max(Ms), stream=stream))
         del W0, A0, B0
+    if not args.no_prefetch:
+        # every layer names the one that runs after it (the last one the first,
+        # which the next batch size starts with): cross-layer L2 prefetch hint
+        for i, lin in enumerate(layers):
+            lin.set_next(layers[(i + 1) % L])
     torch.cuda.synchronize(dev)
 
     xs = {M: make_x(M, K, seed=0).to(dev) for M in Ms}
@@ -364,6 +369,8 @@ def run_ours(args, rank, world, local_rank):
                              f"({L} distinct packed layers, {packed_bytes(K, N, r) * L / 1e6:.0f} MB, "
                              f"plus activations) > 126 MB",
                        "graph": "one CUDA graph per step, kernels chained with programmatic dependent launch",
+                       "prefetch": "off" if args.no_prefetch else
+                                   "each layer's decode kernel reads the next layer's codes from HBM into L2",
                        "dispatch": "tuned (spear_w4ec_tune per layer and M)" if args.tune else "library default",
                        "paths": {str(M): path_name(layers[0].dispatch(M)) for M in Ms},
                        "parallelism": f"replicas x{world}"},
@@ -479,6 +486,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=0, help="layers in the stack (0: enough to exceed 3x L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefetch", action="store_true",
+                    help="do not chain the layers with the cross-layer L2 prefetch hint")
     ap.add_argument("--tune", action="store_true",
                     help="time every path per layer and M first (spear_w4ec_tune); the default dispatch is the "
                          "library's rule, which a profiler cannot perturb")

@@ -141,6 +141,22 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
  * tiles fill at most half of the SMs). */
 int spear_w4ec_dispatch(const spear_w4ec *h, int64_t M, uint32_t *choice);
 
+/* Cross-layer weight prefetch, a hint for serving loops that run a fixed
+ * sequence of layers (the SPEAR pages do not describe one).  `next` names the
+ * layer whose forward follows h's forward on the same stream (h itself is
+ * allowed; NULL clears the hint).  While h's decode-size kernel computes, its
+ * CTAs read next's int4 codes from HBM into the L2 cache once their own codes
+ * have landed, so that next's kernel finds its weights in L2: the weight
+ * stream of one layer overlaps the compute of the layer before.  Results are
+ * identical with or without the hint; a wrong `next` only costs HBM
+ * bandwidth.  The tcgen05 path (more than 32 tokens) ignores it.
+ *   h, next  handles on the same device (SPEAR_ERR_INVALID otherwise)
+ * Destroying `next` clears the hints of every handle that names it.  Not
+ * thread-safe with respect to concurrent calls on the same handles; takes
+ * effect at the next forward (a captured CUDA graph keeps the hint it was
+ * captured with). */
+int spear_w4ec_set_next(spear_w4ec *h, spear_w4ec *next);
+
 /* Per-token gate with no allocation at all, for callers that may not call
  * cudaMalloc (code inside a CUDA graph capture, a real-time serving loop with
  * a fixed memory budget, a host framework whose pool owns every allocation):

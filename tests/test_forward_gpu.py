@@ -165,6 +165,28 @@ def test_invariants_determinism_scaling_permutation():
     P.close()
 
 
+@pytest.mark.parametrize("M,K,N,r", [(1, 4096, 4096, 32), (16, 4096, 4096, 32), (24, 4096, 4096, 32),
+                                     (1, 4096, 14336, 64), (5, 1032, 264, 20)])
+def test_prefetch_hint_leaves_results_unchanged(M, K, N, r):
+    """The cross-layer prefetch hint only moves weights into L2: a chain of
+    layers that name each other (and one that names itself) gives bitwise the
+    same outputs as the same chain without hints; destroying a named layer
+    clears the hint of the layer that names it."""
+    P = Problem(M, K, N, r, seed=M + N)
+    Q = Problem(M, K, N, r, seed=M + N + 1)
+    ref_p, ref_q = _run(P), _run(Q)
+    P.lin.set_next(Q.lin)
+    Q.lin.set_next(P.lin)
+    for _ in range(2):
+        assert torch.equal(_run(P), ref_p)
+        assert torch.equal(_run(Q), ref_q)
+    Q.lin.set_next(Q.lin)
+    assert torch.equal(_run(Q), ref_q)
+    Q.close()
+    assert torch.equal(_run(P), ref_p)   # P's hint was cleared with Q
+    P.close()
+
+
 def test_host_buffer_entry_matches_device_entry():
     from w4_gemm_error_b200 import spear
     P = Problem(9, 1024, 512, 16, seed=9)

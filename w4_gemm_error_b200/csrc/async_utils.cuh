@@ -66,6 +66,23 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 }
 constexpr uint32_t kWaitSleepNs = 1u << 20;   // about a millisecond per suspended try
 
+// Cross-layer weight prefetch: this CTA's share of [base, base + bytes) (a
+// multiple of 16 bytes, 16-byte aligned) read from HBM into L2, in pieces of
+// at most 32 KB.  A hint: nothing waits for it.
+__device__ __forceinline__ void prefetch_l2_share(const void *base, uint64_t bytes)
+{
+    if (!base || bytes == 0)
+        return;
+    const uint64_t units = bytes / 16, per = (units + gridDim.x - 1) / gridDim.x;
+    const uint64_t lo = (uint64_t)blockIdx.x * per * 16;
+    const uint64_t hi = lo + per * 16 < bytes ? lo + per * 16 : bytes;
+    for (uint64_t a = lo; a < hi; a += 32768) {
+        const uint32_t n = (uint32_t)(hi - a < 32768 ? hi - a : 32768);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(static_cast<const char *>(base) + a), "r"(n)
+                     : "memory");
+    }
+}
+
 __device__ __forceinline__ unsigned long long globaltimer()
 {
     unsigned long long t;

@@ -88,6 +88,8 @@ struct DecodeParams {
     int push;             // partial tiles pushed into receive slots of the first CTA
     int x3, g3;           // activations / G rows as one 3-D box per stage (else four 2-D boxes)
     float b_g;
+    const void *pf;       // codes of the next layer, prefetched into L2 (null for none)
+    uint64_t pf_bytes;
 };
 
 // Bytes of one ring stage: the codes of 64 rows x 256 k (or 16 G rows x
@@ -275,6 +277,9 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                     prev ^= 1u;
                 }
             }
+            // every chunk of this CTA is requested: its share of the next layer's
+            // codes goes from HBM into L2 while the consumers finish
+            prefetch_l2_share(p.pf, p.pf_bytes);
         }
         __syncwarp();
     } else if (!is_u) {
@@ -781,7 +786,7 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     // up to 16 tokens on a layer whose 16-row slices fit in shared memory: one
     // CTA per 16 rows over the whole of K, no exchange between CTAs
     if (m->rows && decode_rows_fits(pk, M, num_sms))
-        return launch_decode_rows(pk, m->rows, x, y, M, ec, w.ws_u, w.flags, status, st, num_sms);
+        return launch_decode_rows(pk, m->rows, x, y, M, ec, w, status, st, num_sms);
     const bool use_ec = ec && pk.r > 0;
     DecodeParams p;
     p.Bt = pk.Bt;
@@ -806,6 +811,8 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     p.rp = use_ec ? pk.rp : 0;
     p.R1p = use_ec ? pk.R1p : 0;
     p.b_g = pk.b_g;
+    p.pf = w.pf;
+    p.pf_bytes = w.pf_bytes;
     const int T = M <= 8 ? 1 : (M <= 16 ? 2 : 4);
     // the activations of one stage (TOK rows x 256 k) as one box of the view
     // [k block][token][64 k] when K is a multiple of 64 (then no box reads past

@@ -71,6 +71,8 @@ struct RowsParams {
     uint32_t xs_off;      // byte offset of the staged activations
     int xstage;           // the activations are staged in shared memory (a few tokens)
     float b_g;
+    const void *pf;       // codes of the next layer, prefetched into L2 (null for none)
+    uint64_t pf_bytes;
 };
 
 __device__ __forceinline__ void named_bar_sync(int id, int n)
@@ -372,7 +374,16 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             }
         }
     } else {
-        // ---- spare warp of a row CTA: fetch u while the others compute
+        // ---- spare warp: once this CTA's codes have landed, its share of the next
+        // layer's codes goes from HBM into L2 (the copies no longer compete with
+        // this layer's own); no copy may still be landing when the CTA leaves
+        if (lane == 0) {
+            for (int b = 0; b < nbox; ++b)
+                mbar_wait_bounded(smem_addr(&bars[b]), 0);
+            prefetch_l2_share(p.pf, p.pf_bytes);
+        }
+        __syncwarp();
+        // then, in a row CTA, fetch u while the others compute
         if (!is_u && p.JB > 0) {
             pdl_wait();   // the previous forward has reset the counters
             int good = 1;
@@ -426,11 +437,6 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             }
             named_bar_arrive(1, 32 + kEpi);
         }
-        // no copy may still be landing when the CTA leaves (immediate: every box
-        // has been waited for by a consumer warp, unless a wait gave up)
-        if (lane == 0)
-            for (int b = 0; b < nbox; ++b)
-                mbar_wait_bounded(smem_addr(&bars[b]), 0);
     }
 }
 
@@ -523,7 +529,7 @@ cudaError_t decode_rows_prepare(const Packed &pk, void **maps)
 void decode_rows_free(void *maps) { delete static_cast<RowsMaps *>(maps); }
 
 cudaError_t launch_decode_rows(const Packed &pk, const void *maps, const void *x, void *y, int64_t M, bool ec,
-                               float *ws_u, unsigned *flags, int *status, cudaStream_t st, int num_sms)
+                               const DecodeWork &w, int *status, cudaStream_t st, int num_sms)
 {
     if (!decode_rows_fits(pk, M, num_sms) || !maps)
         return cudaErrorInvalidValue;
@@ -535,8 +541,8 @@ cudaError_t launch_decode_rows(const Packed &pk, const void *maps, const void *x
     p.s = pk.s;
     p.z = pk.z;
     p.y = static_cast<uint16_t *>(y);
-    p.ws_u = ws_u;
-    p.flags = flags;
+    p.ws_u = w.ws_u;
+    p.flags = w.flags;
     p.status = status;
     p.M = M;
     p.N = pk.N;
@@ -560,6 +566,8 @@ cudaError_t launch_decode_rows(const Packed &pk, const void *maps, const void *x
     p.xs_off = pl.xs_off;
     p.xstage = pl.xstage;
     p.b_g = pk.b_g;
+    p.pf = w.pf;
+    p.pf_bytes = w.pf_bytes;
     if (p.nbox > kMaxBoxes || p.ngbox > kMaxBoxes)
         return cudaErrorInvalidValue;
     const int T = pl.T;

@@ -68,6 +68,10 @@ struct DecodeWork {
     void *maps;           // tensor maps of the packed operands (host memory)
     float *ws_u;          // [8][R1p][32] published partials of the EC down-projection
     unsigned *flags;      // two counters, zero between calls
+    // codes of the layer that runs next (prefetched into L2 by the decode
+    // kernels once their own codes have landed), null for none
+    const void *pf;
+    size_t pf_bytes;
 };
 constexpr int kDecodeMaxTokens = 32;   // tokens per launch
 bool decode_supported(const Packed &pk, int num_sms);
@@ -80,13 +84,13 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
 // ---- decode kernel with one CTA per 16 weight rows over the whole of K (up to
 // 16 tokens, K a multiple of 64 and at most 8192, a grid of one wave of two
 // CTAs per SM); launch_decode takes it when it fits.  `maps` is filled by
-// decode_rows_prepare; ws_u and flags are the DecodeWork buffers.
+// decode_rows_prepare; it uses the DecodeWork buffers and prefetch hint.
 bool decode_rows_shape(const Packed &pk);
 bool decode_rows_fits(const Packed &pk, int64_t M, int num_sms);
 cudaError_t decode_rows_prepare(const Packed &pk, void **maps);
 void decode_rows_free(void *maps);
 cudaError_t launch_decode_rows(const Packed &pk, const void *maps, const void *x, void *y, int64_t M, bool ec,
-                               float *ws_u, unsigned *flags, int *status, cudaStream_t st, int num_sms);
+                               const DecodeWork &w, int *status, cudaStream_t st, int num_sms);
 
 // ---- split EC: y[t][n] = bf16(y[t][n] + sum_j v[t][j] * Bt[n][j]), v in fp32
 cudaError_t launch_ec_apply(const Packed &pk, const float *vf, void *y, int64_t M, cudaStream_t st);

@@ -39,6 +39,10 @@ struct spear_w4ec {
     // host-side fault injection (SPEAR_FAULT=alloc|launch|timeout)
     bool fault_launch = false;
     bool fault_timeout = false;
+    // cross-layer prefetch hint: the layer that follows this one, and the
+    // handles that name this one as theirs
+    spear_w4ec *next = nullptr;
+    std::vector<spear_w4ec *> prev;
 };
 
 namespace {
@@ -388,8 +392,38 @@ int spear_w4ec_destroy(spear_w4ec *h)
         return SPEAR_OK;
     DeviceGuard guard(h->device);
     cudaDeviceSynchronize();
+    // no handle may go on prefetching this one's memory
+    for (spear_w4ec *p : h->prev)
+        if (p != h) {
+            p->next = nullptr;
+            p->dec.pf = nullptr;
+            p->dec.pf_bytes = 0;
+        }
+    if (h->next && h->next != h) {
+        auto &v = h->next->prev;
+        v.erase(std::remove(v.begin(), v.end(), h), v.end());
+    }
     free_all(h);
     delete h;
+    return SPEAR_OK;
+}
+
+int spear_w4ec_set_next(spear_w4ec *h, spear_w4ec *next)
+{
+    if (!h || (next && next->device != h->device))
+        return SPEAR_ERR_INVALID;
+    if (h->next) {
+        auto &v = h->next->prev;
+        v.erase(std::remove(v.begin(), v.end(), h), v.end());
+    }
+    h->next = next;
+    h->dec.pf = nullptr;
+    h->dec.pf_bytes = 0;
+    if (next) {
+        next->prev.push_back(h);
+        h->dec.pf = next->pk.codes;
+        h->dec.pf_bytes = (size_t)next->pk.Np * (size_t)next->pk.Kp / 2;
+    }
     return SPEAR_OK;
 }
 

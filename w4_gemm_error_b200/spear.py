@@ -32,7 +32,8 @@ SPEAR_FORCE_TC = 16
 
 EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_forward", "spear_w4ec_forward_host",
             "spear_w4ec_destroy", "spear_w4ec_get_packed", "spear_w4ec_get_gate", "spear_w4ec_sync_status",
-            "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_gate_noalloc", "spear_w4ec_strerror")
+            "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_gate_noalloc", "spear_w4ec_set_next",
+            "spear_w4ec_strerror")
 
 
 class SpearError(RuntimeError):
@@ -62,6 +63,7 @@ def _load():
         "spear_w4ec_tune": [P, P, P, i64, P, ctypes.POINTER(u32)],
         "spear_w4ec_dispatch": [P, i64, ctypes.POINTER(u32)],
         "spear_w4ec_gate_noalloc": [P, i64, i64, P, f32, P, P],
+        "spear_w4ec_set_next": [P, P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -156,6 +158,10 @@ def spear_w4ec_dispatch(h: int, M: int) -> int:
     return choice.value
 
 
+def spear_w4ec_set_next(h: int, next_h):
+    _check(_lib.spear_w4ec_set_next(h, next_h), "spear_w4ec_set_next")
+
+
 def spear_w4ec_gate_noalloc(x, M: int, K: int, w_g, b_g: float, g, stream=None):
     """Gate g[t] for M <= 4096 tokens with no allocation (static scratch inside the library)."""
     _check(_lib.spear_w4ec_gate_noalloc(_ptr(x), M, K, _ptr(w_g), float(b_g), _ptr(g), _stream(stream)),
@@ -219,6 +225,11 @@ class W4ECLinear:
 
     def dispatch(self, M: int) -> int:
         return spear_w4ec_dispatch(self.h, M)
+
+    def set_next(self, other: "W4ECLinear | None"):
+        """Name the layer whose forward follows this one (prefetch hint; None clears)."""
+        spear_w4ec_set_next(self.h, other.h if other is not None else None)
+        self._next = other   # keeps it alive while named
 
     def close(self):
         if getattr(self, "h", None):
