@@ -187,6 +187,32 @@ def test_prefetch_hint_leaves_results_unchanged(M, K, N, r):
     P.close()
 
 
+@pytest.mark.parametrize("M,K,N,r", [(1, 4096, 4096, 32), (4, 4096, 4096, 32), (16, 4096, 4096, 32),
+                                     (1, 4096, 14336, 64)])
+def test_alternating_inputs_and_layers(M, K, N, r):
+    """Forwards whose inputs change from call to call, interleaved over two
+    layers: each output must match the oracle for its own input, so no EC
+    value or partial product left in shared or global memory by an earlier
+    forward (of this layer or another) can stand in for the current one."""
+    import oracle as orc
+    from w4_gemm_error_b200.inputs import make_x
+    P = Problem(M, K, N, r, seed=3)
+    Q = Problem(M, K, N, r, seed=4)
+    xs = [make_x(M, K, seed=100 + i) for i in range(3)]
+    refs = {}
+    for name, prob in (("P", P), ("Q", Q)):
+        codes, s_, z = prob.oracle_packed()
+        L = prob.layer
+        refs[name] = [orc.forward(x, codes, s_, z, L.A, L.B, L.wg, L.b_g) for x in xs]
+    for rnd in range(2):
+        for i, x in enumerate(xs):
+            for name, prob in (("P", P), ("Q", Q)):
+                y = _run(prob, 0, x=x.cuda())
+                assert_close(y, refs[name][i], f"{name} input {i} round {rnd}")
+    P.close()
+    Q.close()
+
+
 def test_host_buffer_entry_matches_device_entry():
     from w4_gemm_error_b200 import spear
     P = Problem(9, 1024, 512, 16, seed=9)

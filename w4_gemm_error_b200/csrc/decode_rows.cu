@@ -79,10 +79,6 @@ __device__ __forceinline__ void named_bar_sync(int id, int n)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
-__device__ __forceinline__ void named_bar_arrive(int id, int n)
-{
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 
 // Bounded wait (one thread) until `expected` EC CTAs have published.
 __device__ __forceinline__ bool wait_count(const unsigned *flag, unsigned expected, int *status)
@@ -118,7 +114,7 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     constexpr int kEpi = kRowsPerCta * TOK;   // epilogue threads: (row, token) pairs
     static_assert(kEpi <= kConsumers, "one epilogue thread per output of the CTA");
     extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t bars[kMaxBoxes];
+    __shared__ __align__(8) uint64_t bars[kMaxBoxes + 1];   // code / G boxes, then "u is in shared memory"
 
     pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, gid = lane >> 2, cl = lane & 3;
@@ -142,6 +138,7 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     if (warp == W && lane == 0) {
         for (int b = 0; b < nbox; ++b)
             mbar_init(smem_addr(&bars[b]), 1);
+        mbar_init(smem_addr(&bars[kMaxBoxes]), 1);
         fence_mbarrier_init_cluster();
         // the weights do not depend on earlier kernels: request them all now
         for (int b = 0; b < nbox; ++b) {
@@ -345,9 +342,10 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 for (int w = 1; w < W; ++w)
                     sum += red[w * TOK * kRowsPerCta + tid];
                 float out = s_epi * sum;
-                if (p.JB > 0) {
-                    named_bar_sync(1, 32 + kEpi);   // u is in shared memory (tokens below M)
-                }
+                // u is in shared memory (tokens below M) once the spare warp has
+                // arrived on this barrier (bounded wait)
+                if (p.JB > 0 && !mbar_wait_bounded(smem_addr(&bars[kMaxBoxes]), 0))
+                    atomicOr(p.status, kStatusTimeout);
                 if (p.JB > 0 && t < p.M) {
                     const uint16_t *btrow = bts + row * p.rp;
                     const float *ut = uT + t * p.rp;
@@ -435,9 +433,13 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 const int t = e / (p.rp - p.r), j = p.r + e - t * (p.rp - p.r);
                 uT[t * p.rp + j] = 0.f;
             }
-            named_bar_arrive(1, 32 + kEpi);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&bars[kMaxBoxes]));   // release: the warp's writes of u come first
         }
     }
+    // no warp leaves before the others are done
+    __syncthreads();
 }
 
 template <int T, int W, int MINB>
