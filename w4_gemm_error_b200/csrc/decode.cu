@@ -165,6 +165,9 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t *const bp = smem_raw + (base - raw);
     const bool push = p.push != 0;
+    // a cluster of one CTA sums nothing across CTAs and needs no cluster barrier
+    // (a barrier.cluster wait costs microseconds even when it has nothing to wait for)
+    const bool solo = CS == 1;
     const Smem L = smem_layout<TOK>(p.S, p.rp, push ? CS - 1 : 0, W);
     const uint32_t rank = cluster_ctarank();
     const int cluster = blockIdx.x / CS;
@@ -234,7 +237,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         }
     }
     __syncthreads();
-    if (push)
+    if (push && !solo)
         cluster_arrive_relaxed();   // the receive barrier of the first CTA is initialised
     int issued = 0;                 // producer: chunks whose codes and activations are requested
     if (producer && lane == 0) {
@@ -457,7 +460,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         __syncthreads();
         if (tid == 0)
             red_release_gpu_add(&p.flags[0], 1u);
-        if (push)
+        if (push && !solo)
             cluster_wait();   // pairs with the arrive after the barrier set-up
         return;
     }
@@ -503,7 +506,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         }
     };
     if (push) {
-        cluster_wait();   // every receive barrier of the cluster is initialised
+        if (!solo)
+            cluster_wait();   // every receive barrier of the cluster is initialised
         if (rank != 0) {
             const uint32_t dst = map_to_rank(base + L.recv + (rank - 1) * (kRows * TOK * 4), 0);
             const uint32_t rbar = map_to_rank(bar_recv, 0);
@@ -515,7 +519,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         }
         if (!fetcher && !poller && CS > 1 && !wait_bounded(bar_recv, 0) && tid == 0)
             atomicOr(p.status, kStatusTimeout);
-        cluster_arrive();     // the tiles have landed: the other CTAs may leave
+        if (!solo)
+            cluster_arrive();     // the tiles have landed: the other CTAs may leave
         if (fetcher || poller) {
             int good = 1;
             if (lane == 0)
@@ -540,7 +545,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 reinterpret_cast<float4 *>(red)[e4] = s;
             }
     } else {
-        cluster_sync();
+        if (!solo)
+            cluster_sync();
         if (fetcher || poller) {
             int good = 1;
             if (lane == 0)
@@ -572,7 +578,8 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             }
         }
         __syncwarp();
-        cluster_sync();  // the other CTAs' shared memory is no longer read
+        if (!solo)
+            cluster_sync();  // the other CTAs' shared memory is no longer read
         if (rank != 0)
             return;
     }
@@ -641,7 +648,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
                 p.y[(int64_t)t * p.N + n] = __bfloat16_as_ushort(__float2bfloat16_rn(out[i]));
         }
     }
-    if (push)
+    if (push && !solo)
         cluster_wait();
 }
 
