@@ -81,14 +81,24 @@ def packed_bytes(K, N, r):
 # profiles/ give the commands.  Reported only while those sources are unchanged.
 TRAFFIC = {
     "decode_qo_4096x4096_r32": dict(
-        kernel="decode_w4ec_kernel",
-        files=("decode.cu", "async_utils.cuh", "device_utils.cuh", "kernels.h"), sha="6f817795c9c902f2",
-        bytes={1: 9.1384e6, 4: 9.1622e6, 16: 9.2541e6},
-        profile="profiles/decode_w4ec_kernel_decode_qo_4096x4096_r32.md"),
+        kernel="decode_rows_kernel",
+        files=('decode_rows.cu', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="6dd6803601107435",
+        bytes={1: 9.1309e6, 4: 9.1556e6, 16: 9.2525e6},
+        profile="profiles/decode_rows_kernel_decode_qo_4096x4096_r32.md"),
+    "decode_mlp_gateup_4096x14336_r64": dict(
+        kernel="decode_w4ec_kernel (1, 16 tokens), tc_w4ec_kernel (64, 128 tokens)",
+        files=('decode.cu', 'tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="1eea718a04bd6fa1",
+        bytes={1: 31.9959e6, 16: 32.1169e6, 64: 33.6867e6, 128: 34.2269e6},
+        profile="profiles/decode_w4ec_kernel_decode_mlp_4096x14336_r64.md"),
+    "decode_mlp_down_14336x4096_r64": dict(
+        kernel="decode_w4ec_kernel (1, 16 tokens), tc_w4ec_kernel (64, 128 tokens)",
+        files=('decode.cu', 'tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="1eea718a04bd6fa1",
+        bytes={1: 32.3018e6, 16: 32.7268e6, 64: 32.3241e6, 128: 34.1788e6},
+        profile="profiles/decode_w4ec_kernel_decode_mlp_4096x14336_r64.md"),
     "prefill_mlp_4096x14336_r64": dict(
         kernel="tc_w4ec_kernel",
-        files=("tc_gemm.cu", "tc_gemm.h", "async_utils.cuh", "device_utils.cuh"), sha="8bd9d2d44fbdf6c0",
-        bytes={2048: 69.713e6, 4096: 155.376e6},
+        files=('tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh'), sha="e9ba96549e58c11d",
+        bytes={2048: 69.5745e6, 4096: 156.0896e6},
         profile="profiles/tc_w4ec_kernel_prefill_mlp_4096x14336_r64.md"),
 }
 
@@ -332,7 +342,9 @@ def run_ours(args, rank, world, local_rank):
         roof = {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": peaks["hbm"], "unit": "GB/s",
                 "frac": round(per_gpu / peaks["hbm"], 4), "traffic": traffic_per_launch(args.workload, Ms),
                 "alg_bytes_per_launch": round(sum(alg_bytes(M, K, N, r) for M in Ms) / len(Ms)),
-                "kernel": "decode_w4ec_kernel (one launch per forward): per-forward time in the chained stack",
+                "kernel": TRAFFIC.get(args.workload, {}).get("kernel", "decode kernels") +
+                          ": per-forward time in the stack (one decode launch per forward; at 64 and 128 "
+                          "tokens the tcgen05 kernel and its prepass)",
                 "peak_source": peaks["source"]}
     else:
         pk = peaks["bf16_sustained"]
