@@ -236,10 +236,11 @@ decode_rows_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         const int sb0 = warp * nsb_cta / W, sb1 = (warp + 1) * nsb_cta / W;
         pdl_wait();
         bool ok = true;
-        if (p.xstage) {
-            // A few tokens: the CTA's activations x[t][kbase .. kbase + 64 nsb_cta)
-            // are staged in shared memory first, one round trip for all of them
-            // (rows padded by 16 bytes to spread them over the banks).
+        if (p.xstage && !is_u) {
+            // A few tokens: the row CTA's activations x[t][0 .. K) are staged in
+            // shared memory first, one round trip for all of them (rows padded by
+            // 16 bytes to spread them over the banks).  A CTA of u (one sub-block
+            // per warp) reads its own directly and saves the staging barrier.
             const int xst = nsb_cta * 64 + 8;
             uint16_t *const xs = reinterpret_cast<uint16_t *>(bp + p.xs_off);
             const int mrows = p.M < TOK ? (int)p.M : TOK;
