@@ -213,6 +213,57 @@ def test_alternating_inputs_and_layers(M, K, N, r):
     Q.close()
 
 
+@pytest.mark.parametrize("M", [1, 4, 16, 24, 64])
+def test_chained_layers_on_one_stream(M):
+    """Four square layers chained on one stream with no host synchronisation
+    in between (each kernel starts early through programmatic dependent launch
+    and waits for its input on the device), in a captured CUDA graph as the
+    bench runs them: every layer's output matches the oracle applied to the
+    input that layer actually received."""
+    import oracle as orc
+    from w4_gemm_error_b200.inputs import make_layer
+    from w4_gemm_error_b200.spear import W4ECLinear
+    K = 1024
+    layers, lins = [], []
+    for i in range(4):
+        L = make_layer(K, K, 32, seed=20 + i)
+        layers.append(L)
+        lins.append(W4ECLinear(L.W.cuda(), L.A.cuda(), L.B.cuda(), L.wg.cuda(), L.b_g, max_M=M))
+    for i in range(4):
+        lins[i].set_next(lins[(i + 1) % 4])
+    P0 = Problem(M, K, K, 32, seed=30)
+    st = torch.cuda.Stream()
+    ys = [torch.empty((M, K), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+
+    def chain():
+        x = P0.xd
+        for i in range(4):
+            lins[i].forward(x, 0, out=ys[i], stream=st)
+            x = ys[i]
+
+    torch.cuda.synchronize()
+    with torch.cuda.stream(st):
+        chain()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            chain()
+        for _ in range(3):
+            g.replay()
+    torch.cuda.synchronize()
+    for lin in lins:
+        assert lin.status() == 0
+    x_in = P0.x
+    for i in range(4):
+        codes, s_, z = orc.pack(layers[i].W)
+        L = layers[i]
+        ref = orc.forward(x_in, codes, s_, z, L.A, L.B, L.wg, L.b_g)
+        assert_close(ys[i], ref, f"layer {i}")
+        x_in = ys[i].cpu()
+    for lin in lins:
+        lin.close()
+    P0.close()
+
+
 def test_host_buffer_entry_matches_device_entry():
     from w4_gemm_error_b200 import spear
     P = Problem(9, 1024, 512, 16, seed=9)
