@@ -16,6 +16,7 @@
 // tile to arrive (no floating-point atomics, run-to-run identical).
 #include <algorithm>
 
+#include "async_utils.cuh"
 #include "device_utils.cuh"
 #include "kernels.h"
 
@@ -37,13 +38,16 @@ struct PrepassParams {
     float *g;
     float *part;
     unsigned *counters;
+    unsigned *ready;   // counted (release) once per token tile when its v is written; null for none
 };
 
 template <int MT>
 __global__ void __launch_bounds__(128) prepass_kernel(PrepassParams p)
 {
-    pdl_launch_dependents();
     pdl_wait();  // x is written by the previous kernel in the stream
+    // the next kernel may start now: x is complete (a tcgen05 kernel that starts
+    // early reads it without waiting)
+    pdl_launch_dependents();
     extern __shared__ float4 smem_f4[];
     float *red = reinterpret_cast<float *>(smem_f4);  // [4][R1p][kTok]
     __shared__ int s_last;
@@ -171,6 +175,11 @@ __global__ void __launch_bounds__(128) prepass_kernel(PrepassParams p)
         const float val = (j < p.r) ? s_gate[tt] * red[(1 + j) * kTok + tt] : 0.f;
         p.v[t * p.rp + j] = p.tf32 ? to_tf32(val) : val;
     }
+    if (p.ready) {
+        __syncthreads();
+        if (tid == 0)
+            red_release_gpu_add(p.ready, 1u);   // this tile's v and g are written
+    }
 }
 
 int pick_splits(int64_t M, int64_t Kp, int num_sms)
@@ -219,7 +228,7 @@ size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms)
 int prepass_counters(int64_t max_M) { return (int)((max_M + kTok - 1) / kTok); }
 
 cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
-                           const PrepassWork &w, cudaStream_t st, int num_sms)
+                           const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready)
 {
     if (M <= 0 || pk.r == 0)
         return cudaSuccess;
@@ -242,6 +251,7 @@ cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v,
     p.g = g;
     p.part = w.part;
     p.counters = w.counters;
+    p.ready = ready;
     const int tiles = (int)((M + kTok - 1) / kTok);
     if (tiles > w.n_counters || (p.S > 1 && (size_t)tiles * p.S * pk.R1p * kTok > w.part_floats))
         return cudaErrorInvalidValue;

@@ -31,6 +31,7 @@ struct spear_w4ec {
     DecodeWork dec{};
     TcWork tc{};
     int *status = nullptr;      // sticky device status bits
+    unsigned *vready = nullptr; // prepass -> tcgen05 kernel: [0] counts of v written, [1] CTAs done
     // staging for forward_host
     void *x_stage = nullptr;
     void *y_stage = nullptr;
@@ -119,6 +120,7 @@ void free_all(spear_w4ec *h)
     decode_free(h->dec);
     tc_free(h->tc);
     cudaFree(h->status);
+    cudaFree(h->vready);
     cudaFree(h->x_stage);
     cudaFree(h->y_stage);
 }
@@ -164,11 +166,19 @@ uint32_t resolve(const spear_w4ec *h, int64_t M, uint32_t flags)
 
 // Gate and v for M tokens: the tcgen05 kernel from 256 tokens on, the
 // split-K mma.sync kernel below that.
-cudaError_t run_prepass(const spear_w4ec *h, const void *x, int64_t M, bool tf32, cudaStream_t st)
+// With `ready`, each CTA (tcgen05) or token tile (mma.sync) counts its v into
+// ready[0]; *expected receives the number of counts.
+cudaError_t run_prepass(const spear_w4ec *h, const void *x, int64_t M, bool tf32, cudaStream_t st,
+                        unsigned *ready = nullptr, unsigned *expected = nullptr)
 {
-    if (M >= 256 && tc_prepass_supported(h->pk))
-        return launch_tc_prepass(h->pk, x, M, h->v, tf32, h->gbuf, h->tc, h->status, st);
-    return launch_prepass(h->pk, x, M, h->v, tf32, h->gbuf, h->pre, st, h->num_sms);
+    if (M >= 256 && tc_prepass_supported(h->pk)) {
+        if (expected)
+            *expected = (unsigned)((M + 127) / 128);
+        return launch_tc_prepass(h->pk, x, M, h->v, tf32, h->gbuf, h->tc, h->status, st, ready);
+    }
+    if (expected)
+        *expected = (unsigned)((M + 15) / 16);
+    return launch_prepass(h->pk, x, M, h->v, tf32, h->gbuf, h->pre, st, h->num_sms, ready);
 }
 
 int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t flags, cudaStream_t st)
@@ -187,16 +197,26 @@ int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t
     const bool decode = (choice & SPEAR_FORCE_DECODE) != 0;
     if (decode && !decode_supported(pk, h->num_sms))
         return SPEAR_ERR_UNSUPPORTED;
-    // the decode kernel computes its own gate and EC down-projection when fused
+    // the decode kernel computes its own gate and EC down-projection when fused;
+    // before the fused tcgen05 kernel, the prepass counts its v into vready so
+    // that the tcgen05 kernel can start its main stages alongside it
+    const bool early = ec && fused && (choice & SPEAR_FORCE_TC) && tc_supported(h);
+    unsigned expected = 0;
     if (ec && !(decode && fused)) {
-        e = run_prepass(h, x, M, (choice & SPEAR_FORCE_TC) != 0 && fused, st);
+        e = run_prepass(h, x, M, (choice & SPEAR_FORCE_TC) != 0 && fused, st, early ? h->vready : nullptr,
+                        &expected);
         if (e != cudaSuccess)
             return from_cuda(e);
     }
     if (choice & SPEAR_FORCE_TC) {
         if (!tc_supported(h))
             return SPEAR_ERR_UNSUPPORTED;
-        e = launch_tc(pk, x, y, M, h->v, ec && fused, h->tc, h->status, h->fault_timeout, st, h->num_sms);
+        e = launch_tc(pk, x, y, M, h->v, ec && fused, h->tc, h->status, h->fault_timeout, st, h->num_sms,
+                      early ? h->vready : nullptr, expected);
+        if (e != cudaSuccess || (early && h->fault_timeout)) {
+            // nothing will reset the prepass's counts: clear them for the next forward
+            cudaMemsetAsync(h->vready, 0, 2 * sizeof(unsigned), st);
+        }
         if (e != cudaSuccess)
             return from_cuda(e);
     } else {
@@ -297,6 +317,7 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r, const s
     chk(alloc_zero(&h->dec.flags, (size_t)2));
     chk(tc_alloc(pk, h->max_M, h->num_sms, h->tc));
     chk(alloc_zero(&h->status, 1));
+    chk(alloc_zero(&h->vready, 2));
     if (e == cudaSuccess)
         e = cudaDeviceSynchronize();
     if (e != cudaSuccess) {

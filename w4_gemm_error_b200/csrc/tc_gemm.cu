@@ -78,6 +78,14 @@ struct TcParams {
     const uint8_t *z;
     uint16_t *y;
     int *status;
+    // early start (fused EC after a prepass): the kernel does not wait for its
+    // predecessor (the prepass, which starts it only once x is complete) before
+    // the main stages; its EC stages wait until v_ready[0] reaches v_expected
+    // (the prepass's release increments), and each CTA waits for the prepass to
+    // finish before it leaves.  The last CTA resets v_ready[0..1].  Null: the
+    // kernel waits for its predecessor first, as usual.
+    unsigned *v_ready;
+    unsigned v_expected;
 };
 
 struct Maps {
@@ -107,6 +115,7 @@ struct PrepassTcParams {
     int tf32;           // round v to tf32
     float *g;           // [M]
     int *status;
+    unsigned *ready;    // counted (release) once this CTA's v is written; null for none
 };
 
 __global__ void __launch_bounds__(PP_THREADS, 1)
@@ -150,14 +159,15 @@ tc_prepass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = tmem_base_slot;
-    // let the next kernel start only now that this CTA holds its tensor memory:
-    // a dependent CTA that cannot allocate then waits for a kernel that needs
-    // nothing from it
-    pdl_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {
             pdl_wait();  // x comes from an earlier kernel in the stream
+            // let the next kernel start only now that x is complete (it may read x
+            // without waiting) and this CTA holds its tensor memory (a dependent
+            // CTA that cannot allocate then waits for a kernel that needs nothing
+            // from it)
+            pdl_launch_dependents();
             int issued = 0;
             for (int kb = 0; kb < p.n_k; ++kb, ++issued) {
                 const uint32_t slot = kb % PP_STAGES, phase = (kb / PP_STAGES) & 1;
@@ -231,6 +241,8 @@ tc_prepass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
 
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && p.ready)
+        red_release_gpu_add(p.ready, 1u);   // this CTA's v and g are written
     if (warp == 1) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(tmem_cols) : "memory");
@@ -296,7 +308,9 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
     if (warp == 0) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            pdl_wait();  // x and v come from earlier kernels in the stream
+            if (!p.v_ready)
+                pdl_wait();  // x and v come from earlier kernels in the stream
+            bool v_seen = p.v_ready == nullptr;
             uint32_t g = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
@@ -321,6 +335,24 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         tma_load_4d(sb + A_BYTES + B_BYTES + C_BYTES / 2, &tm_codes, 0, st & 3, 0, blk + p.kchunks,
                                     full);
                     } else {
+                        if (!v_seen) {
+                            // the prepass has written v for every token (bounded wait);
+                            // the copies below then read it through the async proxy
+                            const long long w0 = clock64();
+                            while (ld_acquire_gpu(p.v_ready) < p.v_expected) {
+                                if (abort_flag || clock64() - w0 > kWaitBudgetCycles) {
+                                    abort_flag = 1;
+                                    atomicOr(p.status, kStatusTimeout);
+                                    ok = false;
+                                    break;
+                                }
+                                __nanosleep(64);
+                            }
+                            if (!ok)
+                                break;
+                            asm volatile("fence.proxy.async;" ::: "memory");
+                            v_seen = true;
+                        }
                         const int e = st - p.n_main;   // 32 tf32 values of j per EC stage
                         mbar_expect_tx(full, A_BYTES + B_BYTES);
                         tma_load_2d(sb, &tm_bt, e * 32, n0, full);
@@ -333,6 +365,10 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                 const uint32_t gg = g - 1 - k, slot = gg % STAGES, phase = (gg / STAGES) & 1;
                 mbar_wait_final(full0 + 8 * slot, phase);
             }
+            // early start: this grid completes only after its predecessor (the
+            // prepass), so that the next kernel's wait still covers both
+            if (p.v_ready)
+                pdl_wait();
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -529,6 +565,11 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
                      : "memory");
     }
+    if (tid == 0 && p.v_ready && atomicAdd(p.v_ready + 1, 1u) == gridDim.x - 1) {
+        // every CTA is past its wait for v and the prepass has finished: reset
+        p.v_ready[0] = 0u;
+        p.v_ready[1] = 0u;
+    }
 }
 
 }  // namespace
@@ -599,7 +640,8 @@ cudaError_t tc_prepare(const Packed &pk, TcWork &w)
 }
 
 cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const float *v, bool ec,
-                      const TcWork &w, int *status, bool zero_wait_budget, cudaStream_t st, int num_sms)
+                      const TcWork &w, int *status, bool zero_wait_budget, cudaStream_t st, int num_sms,
+                      unsigned *v_ready, unsigned v_expected)
 {
     if (M <= 0)
         return cudaSuccess;
@@ -650,6 +692,8 @@ cudaError_t launch_tc(const Packed &pk, const void *x, void *y, int64_t M, const
     p.z = pk.z;
     p.y = static_cast<uint16_t *>(y);
     p.status = status;
+    p.v_ready = use_ec ? v_ready : nullptr;
+    p.v_expected = v_expected;
 
     const void *fn = BN == 32 ? reinterpret_cast<const void *>(tc_w4ec_kernel<32>)
                    : BN == 64 ? reinterpret_cast<const void *>(tc_w4ec_kernel<64>)
@@ -685,7 +729,7 @@ namespace spear {
 bool tc_prepass_supported(const Packed &pk) { return pk.r > 0 && pk.R1p <= 256 && tensor_maps_available(); }
 
 cudaError_t launch_tc_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
-                              const TcWork &w, int *status, cudaStream_t st)
+                              const TcWork &w, int *status, cudaStream_t st, unsigned *ready)
 {
     if (M <= 0)
         return cudaSuccess;
@@ -708,6 +752,7 @@ cudaError_t launch_tc_prepass(const Packed &pk, const void *x, int64_t M, float 
     p.tf32 = tf32 ? 1 : 0;
     p.g = g;
     p.status = status;
+    p.ready = ready;
     const uint32_t stage = 128 * 128 + (((uint32_t)pk.R1p * 128 + 1023u) & ~1023u);
     const size_t smem = (size_t)PP_STAGES * stage + 1024;
     e = raise_smem_limit(reinterpret_cast<const void *>(tc_prepass_kernel), smem);
