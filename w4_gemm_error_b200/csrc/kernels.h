@@ -57,9 +57,10 @@ struct PrepassWork {
     int n_counters;
 };
 // `ready` (may be null): counted (release) once per 16-token tile when its v is
-// written, ceil(M / 16) counts in all.
+// written, ceil(M / 16) counts in all.  `slim`: the register-capped form, whose
+// CTAs fit beside those of a tcgen05 kernel with 64-token tiles.
 cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
-                           const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready);
+                           const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready, bool slim);
 size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms);
 int prepass_counters(int64_t max_M);
 

@@ -41,8 +41,12 @@ struct PrepassParams {
     unsigned *ready;   // counted (release) once per token tile when its v is written; null for none
 };
 
-template <int MT>
-__global__ void __launch_bounds__(128) prepass_kernel(PrepassParams p)
+// MINB = 7 caps the registers at 72 per thread, so that a CTA fits on an SM
+// beside a tcgen05 kernel CTA with 64-token tiles (22 warps of 80 registers,
+// about 200 KB of shared memory) at the price of some spills; MINB = 1 is the
+// fast form for a prepass that runs alone.
+template <int MT, int MINB>
+__global__ void __launch_bounds__(128, MINB) prepass_kernel(PrepassParams p)
 {
     pdl_wait();  // x is written by the previous kernel in the stream
     // the next kernel may start now: x is complete (a tcgen05 kernel that starts
@@ -192,21 +196,23 @@ int pick_splits(int64_t M, int64_t Kp, int num_sms)
 }
 
 using PrepassFn = void (*)(PrepassParams);
-PrepassFn prepass_fn(int MT)
+template <int MINB>
+PrepassFn prepass_fn_b(int MT)
 {
     switch (MT) {
-    case 1: return prepass_kernel<1>;
-    case 2: return prepass_kernel<2>;
-    case 3: return prepass_kernel<3>;
-    case 4: return prepass_kernel<4>;
-    case 5: return prepass_kernel<5>;
-    case 6: return prepass_kernel<6>;
-    case 7: return prepass_kernel<7>;
-    case 8: return prepass_kernel<8>;
-    case 9: return prepass_kernel<9>;
+    case 1: return prepass_kernel<1, MINB>;
+    case 2: return prepass_kernel<2, MINB>;
+    case 3: return prepass_kernel<3, MINB>;
+    case 4: return prepass_kernel<4, MINB>;
+    case 5: return prepass_kernel<5, MINB>;
+    case 6: return prepass_kernel<6, MINB>;
+    case 7: return prepass_kernel<7, MINB>;
+    case 8: return prepass_kernel<8, MINB>;
+    case 9: return prepass_kernel<9, MINB>;
     default: return nullptr;
     }
 }
+PrepassFn prepass_fn(int MT, bool slim) { return slim ? prepass_fn_b<7>(MT) : prepass_fn_b<1>(MT); }
 
 }  // namespace
 
@@ -228,7 +234,7 @@ size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms)
 int prepass_counters(int64_t max_M) { return (int)((max_M + kTok - 1) / kTok); }
 
 cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
-                           const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready)
+                           const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready, bool slim)
 {
     if (M <= 0 || pk.r == 0)
         return cudaSuccess;
@@ -255,7 +261,7 @@ cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v,
     const int tiles = (int)((M + kTok - 1) / kTok);
     if (tiles > w.n_counters || (p.S > 1 && (size_t)tiles * p.S * pk.R1p * kTok > w.part_floats))
         return cudaErrorInvalidValue;
-    PrepassFn fn = prepass_fn(pk.R1p / 16);
+    PrepassFn fn = prepass_fn(pk.R1p / 16, slim);
     if (!fn)
         return cudaErrorInvalidValue;
     const size_t smem = (size_t)4 * pk.R1p * kTok * sizeof(float);

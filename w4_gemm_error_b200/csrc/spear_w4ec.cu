@@ -178,7 +178,9 @@ cudaError_t run_prepass(const spear_w4ec *h, const void *x, int64_t M, bool tf32
     }
     if (expected)
         *expected = (unsigned)((M + 15) / 16);
-    return launch_prepass(h->pk, x, M, h->v, tf32, h->gbuf, h->pre, st, h->num_sms, ready);
+    // beside a tcgen05 kernel with tiles of at most 64 tokens (M <= 64), the
+    // register-capped prepass shares the SMs with it instead of holding them
+    return launch_prepass(h->pk, x, M, h->v, tf32, h->gbuf, h->pre, st, h->num_sms, ready, ready && M <= 64);
 }
 
 int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t flags, cudaStream_t st)
