@@ -82,23 +82,23 @@ def packed_bytes(K, N, r):
 TRAFFIC = {
     "decode_qo_4096x4096_r32": dict(
         kernel="decode_rows_kernel",
-        files=('decode_rows.cu', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="07b61b525eb45229",
-        bytes={1: 9.1311e6, 4: 9.1554e6, 16: 9.2524e6},
+        files=('decode_rows.cu', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="cceab39fd3b7944a",
+        bytes={1: 9.1293e6, 4: 9.1532e6, 16: 9.2512e6},
         profile="profiles/decode_rows_kernel_decode_qo_4096x4096_r32.md"),
     "decode_mlp_gateup_4096x14336_r64": dict(
         kernel="decode_w4ec_kernel (1, 16 tokens), tc_w4ec_kernel (64, 128 tokens)",
-        files=('decode.cu', 'tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="bd3a79d125973742",
-        bytes={1: 31.9959e6, 16: 32.1172e6, 64: 33.6879e6, 128: 34.2281e6},
+        files=('decode.cu', 'tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="cfb6e113f3708182",
+        bytes={1: 31.9955e6, 16: 32.1164e6, 64: 33.6881e6, 128: 34.2278e6},
         profile="profiles/decode_w4ec_kernel_decode_mlp_4096x14336_r64.md"),
     "decode_mlp_down_14336x4096_r64": dict(
         kernel="decode_w4ec_kernel (1, 16 tokens), tc_w4ec_kernel (64, 128 tokens)",
-        files=('decode.cu', 'tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="bd3a79d125973742",
-        bytes={1: 32.3017e6, 16: 32.7265e6, 64: 32.3254e6, 128: 34.1821e6},
+        files=('decode.cu', 'tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="cfb6e113f3708182",
+        bytes={1: 32.3037e6, 16: 32.7282e6, 64: 32.3259e6, 128: 34.1829e6},
         profile="profiles/decode_w4ec_kernel_decode_mlp_4096x14336_r64.md"),
     "prefill_mlp_4096x14336_r64": dict(
         kernel="tc_w4ec_kernel",
         files=('tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh'), sha="d715cce51a6fa3f1",
-        bytes={2048: 69.2401e6, 4096: 155.6396e6},
+        bytes={2048: 69.4048e6, 4096: 154.3288e6},
         profile="profiles/tc_w4ec_kernel_prefill_mlp_4096x14336_r64.md"),
 }
 
