@@ -66,7 +66,10 @@ enum {
     SPEAR_EC_OFF = 1u,        /* drop the EC: the plain W4 GEMM, y = x.W^T */
     SPEAR_FORCE_FUSED = 2u,   /* EC applied inside the GEMM's epilogue / accumulator */
     SPEAR_FORCE_SPLIT = 4u,   /* EC applied by a separate kernel after the GEMM */
-    SPEAR_FORCE_DECODE = 8u,  /* CUDA-core-fed tensor-core split-K kernel (small M) */
+    SPEAR_FORCE_DECODE = 8u,  /* decode kernels, mma.sync on register-dequantised codes (small M):
+                                 one CTA per 16 weight rows over all of K (up to 16 tokens, K a
+                                 multiple of 64 and at most 8192, one wave of CTAs), else the
+                                 split-K streaming kernel (up to 32 tokens per launch) */
     SPEAR_FORCE_TC = 16u      /* tcgen05 / TMEM tile kernel (larger M) */
 };
 
@@ -136,7 +139,7 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
 
 /* The flags (path | fused/split) that forward would use for M tokens now:
  * the tuned choice of M's bucket if spear_w4ec_tune has filled it, else the
- * default rule (fused EC; the decode kernel up to 32 tokens; beyond, the
+ * default rule (fused EC; the decode kernels up to 32 tokens; beyond, the
  * tcgen05 kernel, which splits K for up to 128 tokens on layers whose 128-row
  * tiles fill at most half of the SMs). */
 int spear_w4ec_dispatch(const spear_w4ec *h, int64_t M, uint32_t *choice);
