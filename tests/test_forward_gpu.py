@@ -319,6 +319,15 @@ def test_injected_faults_are_reported(monkeypatch):
         P.lin(P.xd)
     assert ei.value.status == spear.SPEAR_ERR_CUDA
     P.close()
+    # a tcgen05 launch that reports a timeout (its prepass has run and counted
+    # v): the status says so, and the handle's counters are cleared for later
+    monkeypatch.setenv("SPEAR_FAULT", "timeout")
+    P = Problem(64, 512, 256, 8, seed=13)
+    for _ in range(2):
+        torch.cuda.synchronize()
+        P.lin(P.xd, TC | FUSED)
+        assert P.lin.status() == spear.SPEAR_ERR_TIMEOUT
+    P.close()
 
 
 # ------------------------------------------------------------------ tcgen05 tile kernel
