@@ -68,3 +68,5 @@ def test_calls_on_null_handle_are_rejected(lib):
     assert spear.lib().spear_w4ec_forward(None, None, None, 1, 0, None) == spear.SPEAR_ERR_INVALID
     assert spear.lib().spear_w4ec_destroy(None) == spear.SPEAR_OK
     assert spear.lib().spear_w4ec_sync_status(None, None) == spear.SPEAR_ERR_INVALID
+    assert spear.lib().spear_w4ec_set_next(None, None) == spear.SPEAR_ERR_INVALID
+    assert spear.lib().spear_w4ec_dispatch(None, 1, None) == spear.SPEAR_ERR_INVALID
