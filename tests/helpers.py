@@ -69,3 +69,28 @@ class Problem:
 
     def close(self):
         self.lin.close()
+
+
+def tc_token_tile(M: int) -> int:
+    """Token width of the tcgen05 kernel's output tile: the narrowest of 32,
+    64, 128 and 256 that holds M tokens (the tile is 128 weight rows high)."""
+    return 32 if M <= 32 else (64 if M <= 64 else (128 if M <= 128 else 256))
+
+
+def per_tile_samples(M: int, N: int, tile_t: int, tile_n: int = 128, per_tile: int = 4, seed: int = 0):
+    """Output indices (t, n) that hit every tile_t x tile_n output tile at
+    least ``per_tile`` times: the tile's first and last output (clipped to
+    the ragged edge of y) and per_tile - 2 seeded interior ones, so that a
+    tile no launch wrote, or one written with another tile's accumulator,
+    cannot hide between random samples."""
+    rng = np.random.default_rng(seed)
+    ts, ns = [], []
+    for t0 in range(0, M, tile_t):
+        t1 = min(M, t0 + tile_t)
+        for n0 in range(0, N, tile_n):
+            n1 = min(N, n0 + tile_n)
+            ts += [t0, t1 - 1]
+            ns += [n0, n1 - 1]
+            ts += list(rng.integers(t0, t1, per_tile - 2))
+            ns += list(rng.integers(n0, n1, per_tile - 2))
+    return np.asarray(ts, dtype=np.int64), np.asarray(ns, dtype=np.int64)

@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import Problem, assert_close
+from helpers import Problem, assert_close, per_tile_samples, tc_token_tile
 
 pytestmark = pytest.mark.gpu
 
@@ -64,9 +64,12 @@ def test_decode_mlp_full_size(M, K, N):
 def test_decode_mlp_larger_batches_sampled(M, K, N):
     P = Problem(M, K, N, 64, seed=0)
     y = _run(P).cpu()
+    # four outputs of every output tile (the tcgen05 kernel's 128 rows x
+    # 64 / 128 tokens), by index, and 1000 random ones
+    t, n = per_tile_samples(M, N, tc_token_tile(M), seed=M)
     rng = np.random.default_rng(M)
-    t = rng.integers(0, M, 3000)
-    n = rng.integers(0, N, 3000)
+    t = np.concatenate([t, rng.integers(0, M, 1000)])
+    n = np.concatenate([n, rng.integers(0, N, 1000)])
     assert_close(y.float()[t, n], P.oracle_sampled(t, n))
     P.close()
 
@@ -80,12 +83,14 @@ def test_ec_isolated_on_qo_shape():
     ref_off = ref_on - corr
     delta = y_on - y_off
     # Error budget of delta - corr, element by element: the two bf16 roundings
-    # of y (unit roundoff 2^-8 each) and the bf16 rounding of v = g*(x.A)
-    # (2^-8 of each term of sum_j v_j B_j); the main product is computed the
-    # same way with and without the EC, so its fp32 error cancels.
+    # of y (unit roundoff 2^-8 each) and the fp32 evaluation of the correction
+    # (u = x.A accumulated in fp32 from exact bf16 products, then g_t and
+    # sum_j u_j B_j in fp32: far below 1e-4 of sum_j |u_j B_j|); the main
+    # product is computed the same way with and without the EC, so its fp32
+    # error cancels.  No operand of the correction is rounded to bf16.
     xd = P.x.double().numpy()
     terms = g[:, None] * (np.abs(xd @ P.layer.A.double().numpy()) @ np.abs(P.layer.B.double().numpy()))
-    bound = 2.0 ** -8 * (np.abs(ref_on) + np.abs(ref_off) + terms) + 1e-4 * terms + 1e-6
+    bound = 2.0 ** -8 * (np.abs(ref_on) + np.abs(ref_off)) + 1e-4 * terms + 1e-6
     assert np.all(np.abs(delta - corr) <= bound)
     # in aggregate the difference tracks the correction (bf16 rounding of y
     # alone leaves about 10% relative noise at this correction size)
@@ -346,6 +351,38 @@ def test_tc_path_shapes(M, K, N, r):
     P.close()
 
 
+# Persistent tcgen05 kernel with more output tiles than CTAs (148 SMs): each
+# CTA runs two or three tiles in turn, alternating its two TMEM accumulators,
+# reusing them across tiles and carrying the shared-memory ring's phase from
+# one tile to the next.  Every output is compared with the oracle.
+#   1024 x 8192: 4 token tiles x 64 row tiles = 256 tiles
+#   600 x 14336: 3 token tiles (the last one ragged, 88 tokens) x 112 = 336 tiles
+@pytest.mark.parametrize("M,K,N,r", [(1024, 1024, 8192, 32), (600, 512, 14336, 16)])
+def test_tc_persistent_tiles_full_output(M, K, N, r):
+    P = Problem(M, K, N, r, seed=M + 1)
+    tiles = -(-M // tc_token_tile(M)) * (N // 128)
+    assert tiles > torch.cuda.get_device_properties(0).multi_processor_count
+    ref = P.oracle_y()
+    for flags in (TC | FUSED, TC | SPLIT):
+        assert_close(_run(P, flags), ref, f"flags={flags}")
+    assert_close(_run(P, TC | EC_OFF), P.oracle_y(ec_on=False), "EC off")
+    P.close()
+
+
+# Split K at its widest: a layer of 16 row tiles splits every tile's K into
+# min(8, SMs / tiles) = 8 units (128 units on 148 CTAs; the split is sized so
+# that the units never outnumber the SMs), the last unit of each tile summing
+# the partials in split order.  Full outputs, ragged N and ragged tokens.
+@pytest.mark.parametrize("M,K,N,r", [(128, 4096, 2048, 64), (37, 4096, 2000, 32)])
+def test_tc_split_k_eight_ways_full_output(M, K, N, r):
+    P = Problem(M, K, N, r, seed=M + 2)
+    ref = P.oracle_y()
+    for flags in (TC | FUSED, TC | SPLIT):
+        assert_close(_run(P, flags), ref, f"flags={flags}")
+    assert_close(_run(P, TC | EC_OFF), P.oracle_y(ec_on=False), "EC off")
+    P.close()
+
+
 def test_tc_path_invariants():
     P = Problem(300, 1024, 512, 32, seed=13)
     y1 = _run(P, TC)
@@ -392,12 +429,13 @@ def test_tc_ec_isolated():
 
 @pytest.mark.parametrize("M", [2048, 4096])
 def test_prefill_full_size_sampled(M):
-    """Prefill MLP gate/up shape, heavy rows and ~30% open gates: sampled outputs."""
+    """Prefill MLP gate/up shape, heavy rows and ~30% open gates: four outputs
+    of every 128-row x 256-token output tile (896 and 1792 tiles, so every
+    persistent CTA's second and later tiles are among them), by index."""
     P = Problem(M, 4096, 14336, 64, seed=0, w_row_outlier_frac=0.005, gate_open_frac=0.3)
     y = _run(P).float().cpu()
-    rng = np.random.default_rng(M)
-    t = rng.integers(0, M, 2000)
-    n = rng.integers(0, 14336, 2000)
+    t, n = per_tile_samples(M, 14336, tc_token_tile(M), seed=M)
+    assert len(t) == 4 * (M // 256) * 112
     assert_close(y[t, n], P.oracle_sampled(t, n))
     # every row of y is finite and the gate opened for about 30% of tokens
     assert torch.isfinite(y).all()
