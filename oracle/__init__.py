@@ -44,12 +44,13 @@ class _Lib:
         P = ctypes.c_void_p
         i64, i32, f64 = ctypes.c_int64, ctypes.c_int32, ctypes.c_double
         lib.oracle_pack.argtypes = [P, i64, i64, P, P, P]
+        lib.oracle_pack_asym.argtypes = [P, i64, i64, P, P, P]
         lib.oracle_gate.argtypes = [P, i64, i64, P, f64, P]
         lib.oracle_forward.argtypes = [P, i64, i64, i64, i32, P, P, P, P, P, P, f64, i32, P, P, P]
         lib.oracle_forward_sampled.argtypes = [P, i64, i64, i64, i32, P, P, P, P, P, P, f64, i32,
                                                P, P, i64, P]
         lib.oracle_num_threads.argtypes = []
-        for f in (lib.oracle_pack, lib.oracle_gate, lib.oracle_forward,
+        for f in (lib.oracle_pack, lib.oracle_pack_asym, lib.oracle_gate, lib.oracle_forward,
                   lib.oracle_forward_sampled, lib.oracle_num_threads):
             f.restype = ctypes.c_int
         self.lib = lib
@@ -98,6 +99,20 @@ def pack(W, lib=None):
     rc = (lib or _load()).lib.oracle_pack(_ptr(W), N, K, _ptr(codes), _ptr(s), _ptr(z))
     if rc != 0:
         raise ValueError(f"oracle_pack failed ({rc}); K must be a multiple of 8")
+    return codes, s, z
+
+
+def pack_asym(W, lib=None):
+    """Asymmetric (min-max, stored zero point) per-channel int4 of W bf16 [N, K]
+    -> (codes uint32 [N, K/8], s float32 [N], z uint8 [N])."""
+    W = _u16(W)
+    N, K = W.shape
+    codes = np.zeros((N, K // 8), dtype=np.uint32)
+    s = np.zeros(N, dtype=np.float32)
+    z = np.zeros(N, dtype=np.uint8)
+    rc = (lib or _load()).lib.oracle_pack_asym(_ptr(W), N, K, _ptr(codes), _ptr(s), _ptr(z))
+    if rc != 0:
+        raise ValueError(f"oracle_pack_asym failed ({rc}); K must be a multiple of 8")
     return codes, s, z
 
 

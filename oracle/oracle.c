@@ -23,6 +23,14 @@
  *            q    = clamp(c, -8, 7) + 8,  z[n] = 8
  *            an all-zero row has s = 0 and every code 8
  *            code of k = 8j+i sits in bits [4i, 4i+3] of word j of row n
+ *   pack_asym (the same abstract's "state-of-the-art 4-bit quantizers"
+ *            commonly store a per-channel zero point; this is the plain
+ *            min-max form of such a quantiser, with 0 kept in the range)
+ *            lo = min(0, min_k W[n,k]),  hi = max(0, max_k W[n,k])
+ *            s[n] = fp32( fp32(hi - lo) / 15 )
+ *            z[n] = clamp(round_half_even(fp32(-lo / s[n])), 0, 15)
+ *            q    = clamp(round_half_even(fp32(W[n,k] / s[n])) + z[n], 0, 15)
+ *            an all-zero row has s = 0, z = 8 and every code 8
  *   forward  w^[n,k]  = s[n] * (q[n,k] - z[n])
  *            main     = sum_k x[t,k] * w^[n,k]
  *            logit_t  = sum_k x[t,k] * w_g[k] + b_g
@@ -97,6 +105,62 @@ int oracle_pack(const uint16_t *W, int64_t N, int64_t K,
                     if (c > 7.0)
                         c = 7.0;
                     q = (int)c + 8;
+                }
+                word |= (uint32_t)q << (4 * i);
+            }
+            codes[n * words + j] = word;
+        }
+    }
+    return 0;
+}
+
+/* Asymmetric (min-max) per-output-channel round-to-nearest int4 of W [N][K]
+ * into codes [N][K/8], s [N] and a stored zero point z [N] (see the header
+ * comment).  Every fp32 operation is formed in fp64 and rounded once to fp32,
+ * which equals the correctly rounded fp32 operation (fp64 carries more than
+ * 2*24+2 bits, so double rounding of a sum or quotient is innocuous). */
+int oracle_pack_asym(const uint16_t *W, int64_t N, int64_t K,
+                     uint32_t *codes, float *s, uint8_t *z)
+{
+    if (N < 0 || K < 0 || K % 8 != 0)
+        return -1;
+    const int64_t words = K / 8;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const uint16_t *row = W + n * K;
+        double lo = 0.0, hi = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            double w = bf16_to_f64(row[k]);
+            if (w < lo)
+                lo = w;
+            if (w > hi)
+                hi = w;
+        }
+        float range = (float)(hi - lo);
+        float sa = (float)((double)range / 15.0);
+        int zn = 8;
+        if (sa != 0.0f) {
+            double c = nearbyint((double)(float)(-lo / (double)sa));
+            if (c < 0.0)
+                c = 0.0;
+            if (c > 15.0)
+                c = 15.0;
+            zn = (int)c;
+        }
+        s[n] = sa;
+        z[n] = (uint8_t)zn;
+        for (int64_t j = 0; j < words; ++j) {
+            uint32_t word = 0;
+            for (int i = 0; i < 8; ++i) {
+                int q = zn;
+                if (sa != 0.0f) {
+                    float qt = (float)(bf16_to_f64(row[8 * j + i]) / (double)sa);
+                    double c = nearbyint((double)qt) + (double)zn; /* ties to even */
+                    if (c < 0.0)
+                        c = 0.0;
+                    if (c > 15.0)
+                        c = 15.0;
+                    q = (int)c;
                 }
                 word |= (uint32_t)q << (4 * i);
             }

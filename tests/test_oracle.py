@@ -106,6 +106,77 @@ def pin_pack_properties(lib=None):
     assert np.all(np.abs(q[np.arange(64), arg] - 8) == 7)
 
 
+def _read_golden_rows(name):
+    blocks = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if not line:
+                continue
+            key, *vals = line.split()
+            blocks[key] = vals
+    return blocks
+
+
+def pin_pack_asym_golden(lib=None):
+    blocks = _read_golden_rows("pack_asym_rows_k16.txt")
+    names = sorted(k[3:] for k in blocks if k.startswith("row"))
+    W = np.array([[float(v) for v in blocks[f"row{n}"]] for n in names])
+    codes, s, z = oracle.pack_asym(_exact_bf16(W), lib=lib)
+    for i, n in enumerate(names):
+        assert s[i].view(np.uint32) == int(blocks[f"s{n}"][0], 16), f"scale of row {n}"
+        assert int(z[i]) == int(blocks[f"z{n}"][0]), f"zero point of row {n}"
+        assert list(codes[i]) == [int(w, 16) for w in blocks[f"words{n}"]], f"packed words of row {n}"
+        got = [(int(codes[i][k // 8]) >> (4 * (k % 8))) & 0xF for k in range(16)]
+        assert got == [int(c) for c in blocks[f"codes{n}"]], f"codes of row {n}"
+
+
+def pin_asym_requant_identity(lib=None):
+    """W = 2^e (q - z) with a code 0 and a code 15 in every row: the range is
+    exactly 15 * 2^e, so the min-max quantiser gives back s = 2^e, z and q
+    (zero points 0 and 15 included)."""
+    rng = np.random.default_rng(12)
+    N, K = 48, 64
+    q = rng.integers(0, 16, size=(N, K))
+    cols = np.stack([rng.permutation(K)[:2] for _ in range(N)])
+    q[np.arange(N), cols[:, 0]] = 0
+    q[np.arange(N), cols[:, 1]] = 15
+    zp = rng.integers(0, 16, size=N)
+    zp[:2] = (0, 15)
+    e = rng.integers(-10, -1, size=N)
+    W = (q - zp[:, None]).astype(np.float64) * np.exp2(e)[:, None]
+    codes, s, z = oracle.pack_asym(_exact_bf16(W), lib=lib)
+    got = np.stack([(codes[:, k // 8] >> (4 * (k % 8))) & 0xF for k in range(K)], axis=1)
+    assert np.array_equal(got, q)
+    assert np.array_equal(z.astype(np.int64), zp)
+    assert np.array_equal(s.astype(np.float64), np.exp2(e))
+
+
+def pin_asym_properties(lib=None):
+    """Random rows: the range is the min-max one with 0 kept (scale from an
+    IEEE fp32 route of NumPy's own), the zero point maps 0 to a code, and
+    every code is a nearest grid point (within half a step, one ulp of the
+    fp32 quotient allowed) unless the grid's end clips it (within a step)."""
+    rng = np.random.default_rng(6)
+    W = to_bf16(rng.standard_normal((64, 128)) * 0.02 + rng.standard_normal((64, 1)) * 0.01)
+    codes, s, z = oracle.pack_asym(W, lib=lib)
+    Wd = W.double().numpy()
+    lo = np.minimum(Wd.min(axis=1), 0.0).astype(np.float32)
+    hi = np.maximum(Wd.max(axis=1), 0.0).astype(np.float32)
+    assert np.array_equal(s, (hi - lo) / np.float32(15.0))
+    q = np.stack([(codes[:, k // 8] >> (4 * (k % 8))) & 0xF for k in range(128)], axis=1).astype(np.int64)
+    zf = z.astype(np.float64)[:, None]
+    sf = s.astype(np.float64)[:, None]
+    assert np.all(np.abs(-lo.astype(np.float64) / s - z) <= 0.5 + 2.0 ** -18)
+    w_hat = sf * (q - zf)
+    inner = (q > 0) & (q < 15)
+    err = np.abs(Wd - w_hat)
+    assert np.all(err[inner] <= (sf * (0.5 + 2.0 ** -20) + 0 * Wd)[inner])
+    assert np.all(err <= sf * (1.0 + 2.0 ** -20))
+    # both ends of every row are used (the range is the row's own)
+    assert np.all(q.min(axis=1) <= 1) and np.all(q.max(axis=1) >= 14)
+
+
 def pin_forward_golden(lib=None):
     vals = {}
     with open(os.path.join(GOLDEN, "forward_2x8x2_r1.txt")) as f:
@@ -234,7 +305,8 @@ def pin_ec_off_identities(lib=None):
     assert not np.allclose(y_on, y_off)
 
 
-PINS = [pin_pack_golden, pin_requant_identity, pin_pack_properties, pin_forward_golden,
+PINS = [pin_pack_golden, pin_requant_identity, pin_pack_properties, pin_pack_asym_golden,
+        pin_asym_requant_identity, pin_asym_properties, pin_forward_golden,
         pin_bruteforce_exact, pin_gate_closed_forms, pin_gate_closed_matches_matmul,
         pin_gate_open_matches_static_lowrank, pin_rank1_closed_form, pin_ec_off_identities]
 
@@ -277,6 +349,12 @@ MUTANTS = {
     "ties_away_from_zero": ("nearbyint((double)quot)", "round((double)quot)"),
     "scale_over_8": ("amax / 7.0", "amax / 8.0"),
     "fp64_scale_in_quotient": ("/ (double)sn)", "/ (amax / 7.0))"),
+    "asym_range_over_16": ("(double)range / 15.0", "(double)range / 16.0"),
+    "asym_zero_point_sign": ("(-lo / (double)sa)", "(lo / (double)sa)"),
+    "asym_zero_not_in_range": ("double lo = 0.0, hi = 0.0;", "double lo = 1e300, hi = -1e300;"),
+    "asym_ties_away_from_zero": ("nearbyint((double)qt)", "round((double)qt)"),
+    "asym_fp64_quotient": ("float qt = (float)(bf16_to_f64(row[8 * j + i]) / (double)sa);",
+                           "double qt = bf16_to_f64(row[8 * j + i]) / (double)sa;"),
 }
 
 
