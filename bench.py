@@ -1,19 +1,24 @@
 """Benchmark of the W4 + per-token-gated low-rank EC linear layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--workloads all|NAME,...] [--impl ours|reference]
 
 One step is a pass of the whole hot path (gate, EC down-projection, W4 GEMM,
 EC up-projection and combine, dispatch) over a stack of L distinct layers of
-the workload's shape, once for every batch size M of the workload.  For a
-square layer (K == N) the layers are chained (y of one layer is x of the
-next), as in a decode pass through a model; otherwise each layer reads the
-same x.  L is chosen so the packed weights of the stack exceed three times
-the L2 cache (126 MB), so every forward streams its weights from HBM.
+the workload's shape, once for every batch size M of the workload, through
+the library's layer-stack call (spear_w4ec_stack_forward).  For a square
+layer (K == N) the layers are chained (y of one layer is x of the next), as
+in a decode pass through a model; otherwise each layer reads the same x.  L
+is chosen so the packed weights of the stack exceed three times the L2 cache
+(126 MB), so every forward streams its weights from HBM.
 
-Default workload: decode, attention q/o projection, K = N = 4096, rank 32,
-M in {1, 4, 16}: the metric is algorithmic bytes moved per second (GB/s).
-The prefill workload (K = 4096, N = 14336, rank 64, M in {2048, 4096})
-reports TFLOP/s.
+Headline workload (the JSON line's value): decode, attention q/o projection,
+K = N = 4096, rank 32, M in {1, 4, 16}: algorithmic bytes moved per second
+(GB/s).  The same run measures, the same way, the rest of the metric under
+"workloads": the MLP up and down projections at decode batch sizes (GB/s)
+and the prefill MLP shape (K = 4096, N = 14336, rank 64, M in {2048, 4096};
+TFLOP/s).  Each record has its own roofline, EC overhead, end-to-end figure
+(the host-buffer stack call, spear_w4ec_stack_forward_host) and clocks.
 
 Under torchrun every rank runs the same stack on its own GPU (independent
 replicas, no data-path collective: weak scaling); the time is the maximum
@@ -75,45 +80,33 @@ def packed_bytes(K, N, r):
     return N * K // 2 + 5 * N + 2 * K * (r + 1) + 2 * r * N
 
 
-# DRAM bytes (read + write) per launch of each workload's dominant kernel, by
-# batch size, from one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum)
-# of the kernel sources whose SHA-256 prefix is given; the summaries under
-# profiles/ give the commands.  Reported only while those sources are unchanged.
-TRAFFIC = {
-    "decode_qo_4096x4096_r32": dict(
-        kernel="decode_rows_kernel",
-        files=('decode_rows.cu', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="cceab39fd3b7944a",
-        bytes={1: 9.1293e6, 4: 9.1532e6, 16: 9.2512e6},
-        profile="profiles/decode_rows_kernel_decode_qo_4096x4096_r32.md"),
-    "decode_mlp_gateup_4096x14336_r64": dict(
-        kernel="decode_w4ec_kernel (1, 16 tokens), tc_w4ec_kernel (64, 128 tokens)",
-        files=('decode.cu', 'tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="cfb6e113f3708182",
-        bytes={1: 31.9955e6, 16: 32.1164e6, 64: 33.6881e6, 128: 34.2278e6},
-        profile="profiles/decode_w4ec_kernel_decode_mlp_4096x14336_r64.md"),
-    "decode_mlp_down_14336x4096_r64": dict(
-        kernel="decode_w4ec_kernel (1, 16 tokens), tc_w4ec_kernel (64, 128 tokens)",
-        files=('decode.cu', 'tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh', 'kernels.h'), sha="cfb6e113f3708182",
-        bytes={1: 32.3037e6, 16: 32.7282e6, 64: 32.3259e6, 128: 34.1829e6},
-        profile="profiles/decode_w4ec_kernel_decode_mlp_4096x14336_r64.md"),
-    "prefill_mlp_4096x14336_r64": dict(
-        kernel="tc_w4ec_kernel",
-        files=('tc_gemm.cu', 'tc_gemm.h', 'async_utils.cuh', 'device_utils.cuh'), sha="d715cce51a6fa3f1",
-        bytes={2048: 69.4048e6, 4096: 154.3288e6},
-        profile="profiles/tc_w4ec_kernel_prefill_mlp_4096x14336_r64.md"),
-}
+TRAFFIC_FILE = os.path.join(ROOT, "bench_traffic.json")
+
+
+def load_traffic():
+    """Measured DRAM bytes per launch of each workload's dominant kernel (one
+    ncu capture per kernel source state; see bench_traffic.json)."""
+    with open(TRAFFIC_FILE) as f:
+        data = json.load(f)["workloads"]
+    return {name: dict(t, bytes={int(m): float(b) for m, b in t["bytes"].items()}) for name, t in data.items()}
+
+
+def sources_sha(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "w4_gemm_error_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
 
 
 def traffic_per_launch(workload, Ms):
-    """Mean measured DRAM bytes per launch over the step's batch sizes, or None."""
-    import hashlib
-    t = TRAFFIC.get(workload)
+    """Mean measured DRAM bytes per launch over the step's batch sizes, or None
+    (no capture, or the kernel sources changed since it was taken)."""
+    t = load_traffic().get(workload)
     if t is None or any(M not in t["bytes"] for M in Ms):
         return None
-    h = hashlib.sha256()
-    for f in t["files"]:
-        with open(os.path.join(ROOT, "w4_gemm_error_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
-    if h.hexdigest()[:16] != t["sha"]:
+    if sources_sha(t["files"]) != t["sha"]:
         return None
     return round(sum(t["bytes"][M] for M in Ms) / len(Ms))
 
@@ -199,15 +192,25 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(args, rank, world, local_rank):
+def _timed_region_peak(peaks, seconds):
+    """bf16 denominator for a timed region of `seconds`: the burst figure for a
+    region under two seconds, the sustained (power-capped) one for longer."""
+    if seconds < 2.0:
+        return peaks["bf16"], peaks["source"] + " (burst: timed region %.2f s)" % seconds
+    return peaks["bf16_sustained"], peaks["source"] + " (sustained: timed region %.2f s)" % seconds
+
+
+def measure_workload(name, args, rank, world, local_rank, cpu_seconds):
+    """Time one workload on this rank's GPU: the graph-captured stack (EC on and
+    EC off) on device-resident inputs, and the host-buffer stack call end to
+    end.  Returns the rank-0 record (None elsewhere)."""
     import torch
     import torch.distributed as dist
     from w4_gemm_error_b200.inputs import make_layer, make_x
     from w4_gemm_error_b200 import spear
 
-    wl = WORKLOADS[args.workload]
+    wl = WORKLOADS[name]
     K, N, r, Ms = wl["K"], wl["N"], wl["r"], wl["Ms"]
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.Stream(device=dev)
 
@@ -227,31 +230,35 @@ def run_ours(args, rank, world, local_rank):
             B = torch.roll(B0, shifts=31 * i, dims=1).contiguous()
             layers.append(spear.W4ECLinear(W, A, B, wg, base.b_g, max_M=max(Ms), stream=stream))
         del W0, A0, B0
-    if not args.no_prefetch:
-        # every layer names the one that runs after it (the last one the first,
-        # which the next batch size starts with): cross-layer L2 prefetch hint
-        for i, lin in enumerate(layers):
-            lin.set_next(layers[(i + 1) % L])
     torch.cuda.synchronize(dev)
-
-    xs = {M: make_x(M, K, seed=0).to(dev) for M in Ms}
-    bufs = {M: [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(2)] for M in Ms}
     if args.tune:
         # the library's adaptive dispatch: each layer times its legal paths once per batch size
+        xs_t = {M: make_x(M, K, seed=0).to(dev) for M in Ms}
+        y_t = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in Ms}
         with torch.cuda.stream(stream):
             for M in Ms:
                 for lin in layers:
-                    lin.tune(xs[M], bufs[M][0], stream=stream)
+                    lin.tune(xs_t[M], y_t[M], stream=stream)
         torch.cuda.synchronize(dev)
+    # the step's layer sequence as one stack (spear_w4ec_stack_*): chained
+    # (square layers: y of layer l is x of layer l + 1) or all reading x;
+    # intermediates alternate between two buffers; every EC placed
+    ops = []
+    for i, lin in enumerate(layers):
+        src = 0 if (i == 0 or not chain) else 2 + (i - 1) % 2
+        dst = 1 if i == L - 1 else 2 + i % 2
+        ops.append((lin, src, dst, 1))
+    stack = spear.W4ECStack(ops, max(Ms))
+    if args.no_prefetch:
+        for lin in layers:
+            lin.set_next(None)
+
+    xs = {M: make_x(M, K, seed=0).to(dev) for M in Ms}
+    ys = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in Ms}
 
     def step(flags=0):
         for M in Ms:
-            x = xs[M]
-            for i, lin in enumerate(layers):
-                y = bufs[M][i % 2]
-                lin.forward(x, flags, out=y, stream=stream)
-                if chain:
-                    x = y
+            stack.forward(xs[M], flags, out=ys[M], stream=stream)
 
     def capture(flags):
         g = torch.cuda.CUDAGraph()
@@ -291,7 +298,7 @@ def run_ours(args, rank, world, local_rank):
     g_off = capture(spear.SPEAR_EC_OFF)
     ms_on, clocks = timed(g_on, args.steps, args.warmup, sample_clocks=True)
     ms_off, _ = timed(g_off, args.steps, args.warmup)
-    off_steps = args.steps
+    del g_on, g_off
 
     forwards_per_step = L * len(Ms)
     if wl["kind"] == "decode":
@@ -304,26 +311,18 @@ def run_ours(args, rank, world, local_rank):
     value = total_units / (ms_on * 1e-3) / scale
     per_gpu = value / world
     ms_per_step = ms_on / args.steps
-    ec_overhead = (ms_on / args.steps) / (ms_off / off_steps) - 1.0
+    ec_overhead = ms_on / ms_off - 1.0
 
-    # end to end through the public API: pinned host x in, device chain, host y out, per step
+    # end to end through the public C ABI: one host-buffer stack call per batch
+    # size and step (spear_w4ec_stack_forward_host: pinned x in, the layers on
+    # the device, y out, stream synchronised), wall clock
     x_host = {M: make_x(M, K, seed=0).pin_memory() for M in Ms}
     y_host = {M: torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for M in Ms}
-    x_dev = {M: torch.empty((M, K), dtype=torch.bfloat16, device=dev) for M in Ms}
     e2e_steps = max(3, min(args.steps, 50))
 
     def e2e_step():
         for M in Ms:
-            with torch.cuda.stream(stream):
-                x_dev[M].copy_(x_host[M], non_blocking=True)
-                x = x_dev[M]
-                for i, lin in enumerate(layers):
-                    y = bufs[M][i % 2]
-                    lin.forward(x, 0, out=y, stream=stream)
-                    if chain:
-                        x = y
-                y_host[M].copy_(y, non_blocking=True)
-            stream.synchronize()
+            stack.forward_host(x_host[M], y_host[M], stream=stream)
 
     for _ in range(3):
         e2e_step()
@@ -338,21 +337,23 @@ def run_ours(args, rank, world, local_rank):
     d2h = sum(M * N * 2 for M in Ms)
 
     peaks = load_peaks()
+    tr = load_traffic().get(name, {})
     if wl["kind"] == "decode":
         roof = {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": peaks["hbm"], "unit": "GB/s",
-                "frac": round(per_gpu / peaks["hbm"], 4), "traffic": traffic_per_launch(args.workload, Ms),
+                "frac": round(per_gpu / peaks["hbm"], 4), "traffic": traffic_per_launch(name, Ms),
                 "alg_bytes_per_launch": round(sum(alg_bytes(M, K, N, r) for M in Ms) / len(Ms)),
-                "kernel": TRAFFIC.get(args.workload, {}).get("kernel", "decode kernels") +
+                "kernel": tr.get("kernel", "decode kernels") +
                           ": per-forward time in the stack (one decode launch per forward; at 64 and 128 "
                           "tokens the tcgen05 kernel and its prepass)",
-                "peak_source": peaks["source"]}
+                "peak_source": peaks["source"] + " (HBM copy)"}
     else:
-        pk = peaks["bf16_sustained"]
+        pk, src_note = _timed_region_peak(peaks, ms_on * 1e-3)
         roof = {"bound": "tensor", "achieved": round(per_gpu, 1), "peak": pk, "unit": "TFLOP/s",
-                "frac": round(per_gpu / pk, 4), "traffic": traffic_per_launch(args.workload, Ms),
-                "kernel": "tc_w4ec_kernel: per-forward time, which also holds the tc_prepass_kernel launch "
-                          "(about 5% of the launch list), so the kernel's own rate is higher",
-                "peak_source": peaks["source"] + " (sustained)"}
+                "frac": round(per_gpu / pk, 4), "traffic": traffic_per_launch(name, Ms),
+                "alg_flops_per_launch": round(sum(alg_flops(M, K, N, r) for M in Ms) / len(Ms)),
+                "kernel": "tc_w4ec_kernel: per-forward time, which also holds the tc_prepass_kernel launch, "
+                          "so the kernel's own rate is higher",
+                "peak_source": src_note}
 
     launches_per_forward = {}
     for M in Ms:
@@ -366,20 +367,19 @@ def run_ours(args, rank, world, local_rank):
     gpu_launches = args.steps * L * sum(launches_per_forward.values())
 
     # bytes one step touches: every layer's packed weights, each M's input and its output buffers
-    touched = packed_bytes(K, N, r) * L + sum(M * K * 2 + min(L, 2) * M * N * 2 for M in Ms)
+    touched = packed_bytes(K, N, r) * L + sum(M * K * 2 + min(L, 3) * M * N * 2 for M in Ms)
     out = None
     if rank == 0:
-        cpu = cpu_baseline(args, wl) if world == 1 and not args.no_cpu_baseline else None
+        cpu = cpu_baseline(wl, cpu_seconds) if (world == 1 and cpu_seconds > 0) else None
         out = {
-            "metric": METRIC, "value": round(value, 2), "unit": unit, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "M": list(Ms), "K": K, "N": N, "r": r, "layers": L,
+            "value": round(value, 2), "unit": unit, "ms_per_step": round(ms_per_step, 4),
+            "config": {"workload": name, "M": list(Ms), "K": K, "N": N, "r": r, "layers": L,
                        "chained": chain, "forwards_per_step": forwards_per_step,
                        "weights": "int4 per output channel (RTN), A/B/w_g bf16",
                        "l2": f"inputs larger than L2: each step touches {touched / 1e6:.0f} MB "
                              f"({L} distinct packed layers, {packed_bytes(K, N, r) * L / 1e6:.0f} MB, "
                              f"plus activations) > 126 MB",
+                       "api": "spear_w4ec_stack_forward (one stack of the L layers, every EC placed) per M",
                        "graph": "one CUDA graph per step, kernels chained with programmatic dependent launch",
                        "prefetch": "off" if args.no_prefetch else
                                    "each layer's decode kernel reads the next layer's codes from HBM into L2",
@@ -388,12 +388,47 @@ def run_ours(args, rank, world, local_rank):
                        "parallelism": f"replicas x{world}"},
             "ec_overhead": round(ec_overhead, 4),
             "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "api": "spear_w4ec_forward per layer, eager, pinned host I/O"},
+                    "d2h_bytes_per_step": d2h,
+                    "api": "spear_w4ec_stack_forward_host per M (C ABI, pinned host x and y, copies and "
+                           "stream sync inside the timed region)"},
             "roofline": roof, "clocks": clocks, "gpu_launches": gpu_launches,
             "cpu_baseline": cpu,
         }
+    stack.close()
     for lin in layers:
         lin.close()
+    del layers
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    torch.cuda.set_device(local_rank)
+    names = [args.workload]
+    if args.workloads == "all":
+        names += [n for n in WORKLOADS if n != args.workload]
+    elif args.workloads:
+        names += [n for n in args.workloads.split(",") if n and n != args.workload]
+    records = {}
+    for i, name in enumerate(names):
+        if name not in WORKLOADS:
+            raise SystemExit(f"unknown workload {name}")
+        cpu_s = 0.0 if args.no_cpu_baseline else (10.0 if i == 0 else 3.0)
+        records[name] = measure_workload(name, args, rank, world, local_rank, cpu_s)
+    if rank != 0:
+        return None
+    head = records[args.workload]
+    out = {"metric": METRIC, "value": head["value"], "unit": head["unit"], "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": head["config"], "ec_overhead": head["ec_overhead"], "e2e": head["e2e"],
+           "roofline": head["roofline"], "clocks": head["clocks"], "gpu_launches": head["gpu_launches"],
+           "cpu_baseline": head["cpu_baseline"]}
+    if len(names) > 1:
+        # the metric's other half and the other shapes, measured the same way in this process
+        out["workloads"] = {n: records[n] for n in names}
     return out
 
 
@@ -443,7 +478,7 @@ def _run_oracle_sample(wl, lay, codes, s, z, jobs):
     return units
 
 
-def cpu_baseline(args, wl, min_seconds=10.0):
+def cpu_baseline(wl, min_seconds=10.0):
     import oracle
     lay, codes, s, z, jobs = _oracle_sample(wl)
     _run_oracle_sample(wl, lay, codes, s, z, jobs)  # warm
@@ -494,7 +529,11 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="decode_qo_4096x4096_r32", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="decode_qo_4096x4096_r32", choices=sorted(WORKLOADS),
+                    help="the headline workload of the JSON line")
+    ap.add_argument("--workloads", default="all",
+                    help="further workloads measured in the same run and reported under 'workloads' "
+                         "(comma-separated names, 'all' (default) or '' for none)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=0, help="layers in the stack (0: enough to exceed 3x L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

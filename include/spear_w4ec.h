@@ -182,6 +182,69 @@ int spear_w4ec_set_next(spear_w4ec *h, spear_w4ec *next);
 int spear_w4ec_gate_noalloc(const void *x, int64_t M, int64_t K, const void *w_g, float b_g, float *g,
                             void *stream);
 
+/* ---- Layer stack with a caller-given EC placement.
+ *
+ * SPEAR, Abstract: Error Compensators are placed only at the most
+ * error-sensitive layers (its diagnostic that picks them is not part of this
+ * library; the placement is an input here).  A stack runs a fixed sequence
+ * of packed layers on one stream, each op reading one activation buffer and
+ * writing another, so a decoder's projections (q, k, v from h; o from q;
+ * gate and up from o; down from up) or a plain chain of layers run as one
+ * call, with the EC of each op switched on or off by the placement.
+ *
+ * Buffers are numbered: 0 is the stack's input x (read only), 1 its output
+ * y (written by the last op and no other), 2 and up are intermediates the
+ * stack allocates (max_M rows of the widest activation written there).
+ * Every buffer holds [M][width] bf16, row-major and dense. */
+typedef struct spear_w4ec_stack spear_w4ec_stack; /* opaque, owned by the library */
+
+typedef struct spear_w4ec_stack_op {
+    spear_w4ec *layer; /* the packed layer this op runs (not owned by the stack) */
+    int32_t in;        /* buffer it reads: 0 (the input x) or an intermediate >= 2 */
+    int32_t out;       /* buffer it writes: 1 (the output y, last op only) or an intermediate >= 2 */
+    int32_t ec;        /* EC placement: 1 applies the layer's EC (if it has one), 0 runs the
+                          plain W4 GEMM (as SPEAR_EC_OFF) */
+} spear_w4ec_stack_op;
+
+/* Build a stack of n_ops ops (1 <= n_ops <= 4096) for up to max_M tokens.
+ * Checked here, all SPEAR_ERR_INVALID: every layer non-NULL, on one device
+ * and created with max_M at least this max_M; SPEAR_ERR_STATE if a layer is
+ * not packed.  Buffer rules: intermediates are numbered 2 .. n_ops + 1; an op
+ * reads 0 or an intermediate that an earlier op wrote, with the width (N)
+ * that op wrote equal to its own K; every op that reads 0 has the same K;
+ * only the last op writes 1; no op reads the buffer it writes.  The ops are
+ * copied; the layers must outlive the stack.  Allocates the intermediates
+ * and host-call staging buffers (max_M rows each) on the layers' device, and
+ * names each op's layer's successor in the sequence (the last names the
+ * first) as its prefetch hint (spear_w4ec_set_next), replacing earlier hints. */
+int spear_w4ec_stack_create(spear_w4ec_stack **out, const spear_w4ec_stack_op *ops, int32_t n_ops,
+                            int64_t max_M);
+
+/* Run the ops in order on `stream` for M tokens (0 <= M <= max_M; M = 0 is a
+ * no-op): x dev bf16 [M][K of the ops reading 0], y dev bf16 [M][N of the
+ * last op], both 16-byte aligned.  Each op's output equals that of
+ * spear_w4ec_forward on the same input with flags 0 (EC placed) or
+ * SPEAR_EC_OFF (EC not placed), bit for bit.  `flags` (0 for the placement
+ * as given) may add SPEAR_FORCE_* path flags or SPEAR_EC_OFF, which then
+ * apply to every op. */
+int spear_w4ec_stack_forward(spear_w4ec_stack *s, const void *x, void *y, int64_t M, uint32_t flags,
+                             void *stream);
+
+/* The same with x and y in HOST memory: copies x to the stack's device
+ * staging buffer, runs the ops, copies y back, all on `stream`, then
+ * synchronises the stream.  Pinned host memory gives the fastest copies. */
+int spear_w4ec_stack_forward_host(spear_w4ec_stack *s, const void *x_host, void *y_host, int64_t M,
+                                  uint32_t flags, void *stream);
+
+/* Device address of intermediate buffer `index` (>= 2) in *ptr: after a
+ * forward on M tokens it holds the [M][width] output of the last op that
+ * wrote it (for inspection and tests). */
+int spear_w4ec_stack_buffer(const spear_w4ec_stack *s, int32_t index, void **ptr);
+
+/* Free the stack's buffers (synchronises the device first); the layers are
+ * left as they are.  NULL is a no-op. */
+int spear_w4ec_stack_destroy(spear_w4ec_stack *s);
+
 /* Human-readable name of a status code (static storage). */
 const char *spear_w4ec_strerror(int status);
 

@@ -70,3 +70,21 @@ def test_calls_on_null_handle_are_rejected(lib):
     assert spear.lib().spear_w4ec_sync_status(None, None) == spear.SPEAR_ERR_INVALID
     assert spear.lib().spear_w4ec_set_next(None, None) == spear.SPEAR_ERR_INVALID
     assert spear.lib().spear_w4ec_dispatch(None, 1, None) == spear.SPEAR_ERR_INVALID
+
+
+def test_stack_calls_reject_bad_arguments_before_touching_the_device(lib):
+    from w4_gemm_error_b200 import spear
+    L = spear.lib()
+    s = ctypes.c_void_p()
+    assert L.spear_w4ec_stack_create(None, None, 1, 1) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_stack_create(ctypes.byref(s), None, 1, 1) == spear.SPEAR_ERR_INVALID
+    ops = (spear.StackOp * 1)(spear.StackOp(None, 0, 1, 1))
+    assert L.spear_w4ec_stack_create(ctypes.byref(s), ops, 0, 1) == spear.SPEAR_ERR_INVALID   # no op
+    assert L.spear_w4ec_stack_create(ctypes.byref(s), ops, 1, 0) == spear.SPEAR_ERR_INVALID   # max_M < 1
+    assert L.spear_w4ec_stack_create(ctypes.byref(s), ops, 1, 4) == spear.SPEAR_ERR_INVALID   # NULL layer
+    assert s.value is None
+    assert L.spear_w4ec_stack_forward(None, None, None, 1, 0, None) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_stack_forward_host(None, None, None, 1, 0, None) == spear.SPEAR_ERR_INVALID
+    p = ctypes.c_void_p()
+    assert L.spear_w4ec_stack_buffer(None, 2, ctypes.byref(p)) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_stack_destroy(None) == spear.SPEAR_OK

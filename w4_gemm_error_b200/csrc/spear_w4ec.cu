@@ -13,62 +13,14 @@
 
 #include "spear_w4ec.h"
 #include "device_utils.cuh"
+#include "handle.h"
 #include "kernels.h"
 #include "tc_gemm.h"
 
 using namespace spear;
 
-struct spear_w4ec {
-    int device = 0;
-    int num_sms = 148;
-    int64_t max_M = 0;
-    Packed pk{};
-    bool packed = false;
-    // workspace
-    float *v = nullptr;         // [max_M][rp] fp32: g_t * (x . A) (tf32-rounded for the tcgen05 path)
-    float *gbuf = nullptr;      // [max_M] gate values
-    PrepassWork pre{};
-    DecodeWork dec{};
-    TcWork tc{};
-    int *status = nullptr;      // sticky device status bits
-    unsigned *vready = nullptr; // prepass -> tcgen05 kernel: [0] counts of v written, [1] CTAs done
-    // staging for forward_host
-    void *x_stage = nullptr;
-    void *y_stage = nullptr;
-    // dispatch table: flags per M bucket, 0 = not tuned
-    uint32_t table[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
-    // host-side fault injection (SPEAR_FAULT=alloc|launch|timeout)
-    bool fault_launch = false;
-    bool fault_timeout = false;
-    // cross-layer prefetch hint: the layer that follows this one, and the
-    // handles that name this one as theirs
-    spear_w4ec *next = nullptr;
-    std::vector<spear_w4ec *> prev;
-};
-
 namespace {
 
-class DeviceGuard {
-  public:
-    explicit DeviceGuard(int dev)
-    {
-        if (cudaGetDevice(&prev_) != cudaSuccess)
-            prev_ = -1;
-        if (prev_ != dev)
-            ok_ = cudaSetDevice(dev) == cudaSuccess;
-    }
-    ~DeviceGuard()
-    {
-        int cur = -1;
-        if (prev_ >= 0 && cudaGetDevice(&cur) == cudaSuccess && cur != prev_)
-            cudaSetDevice(prev_);
-    }
-    bool ok() const { return ok_; }
-
-  private:
-    int prev_ = -1;
-    bool ok_ = true;
-};
 
 const char *env_fault()
 {
@@ -240,6 +192,17 @@ int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t
 }
 
 }  // namespace
+
+namespace spear {
+
+int status_of(cudaError_t e) { return from_cuda(e); }
+
+int forward_checked(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t flags, cudaStream_t st)
+{
+    return run_forward(h, x, y, M, flags, st);
+}
+
+}  // namespace spear
 
 extern "C" {
 

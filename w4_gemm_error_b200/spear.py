@@ -33,7 +33,8 @@ SPEAR_FORCE_TC = 16
 EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_forward", "spear_w4ec_forward_host",
             "spear_w4ec_destroy", "spear_w4ec_get_packed", "spear_w4ec_get_gate", "spear_w4ec_sync_status",
             "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_gate_noalloc", "spear_w4ec_set_next",
-            "spear_w4ec_strerror")
+            "spear_w4ec_stack_create", "spear_w4ec_stack_forward", "spear_w4ec_stack_forward_host",
+            "spear_w4ec_stack_buffer", "spear_w4ec_stack_destroy", "spear_w4ec_strerror")
 
 
 class SpearError(RuntimeError):
@@ -44,6 +45,13 @@ class SpearError(RuntimeError):
 
 class _Opts(ctypes.Structure):
     _fields_ = [("max_M", ctypes.c_int64), ("device", ctypes.c_int32)]
+
+
+class StackOp(ctypes.Structure):
+    """spear_w4ec_stack_op: the layer handle, the buffers it reads and writes,
+    and whether its EC is placed (1) or not (0)."""
+    _fields_ = [("layer", ctypes.c_void_p), ("in_", ctypes.c_int32), ("out", ctypes.c_int32),
+                ("ec", ctypes.c_int32)]
 
 
 def _load():
@@ -64,6 +72,11 @@ def _load():
         "spear_w4ec_dispatch": [P, i64, ctypes.POINTER(u32)],
         "spear_w4ec_gate_noalloc": [P, i64, i64, P, f32, P, P],
         "spear_w4ec_set_next": [P, P],
+        "spear_w4ec_stack_create": [ctypes.POINTER(P), ctypes.POINTER(StackOp), i32, i64],
+        "spear_w4ec_stack_forward": [P, P, P, i64, u32, P],
+        "spear_w4ec_stack_forward_host": [P, P, P, i64, u32, P],
+        "spear_w4ec_stack_buffer": [P, i32, ctypes.POINTER(P)],
+        "spear_w4ec_stack_destroy": [P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -168,6 +181,33 @@ def spear_w4ec_gate_noalloc(x, M: int, K: int, w_g, b_g: float, g, stream=None):
            "spear_w4ec_gate_noalloc")
 
 
+def spear_w4ec_stack_create(ops, max_M: int) -> int:
+    """ops: sequence of (layer handle, in, out, ec) tuples."""
+    arr = (StackOp * len(ops))(*[StackOp(h, i, o, e) for (h, i, o, e) in ops])
+    s = ctypes.c_void_p()
+    _check(_lib.spear_w4ec_stack_create(ctypes.byref(s), arr, len(ops), max_M), "spear_w4ec_stack_create")
+    return s.value
+
+
+def spear_w4ec_stack_forward(s: int, x, y, M: int, flags: int = 0, stream=None):
+    _check(_lib.spear_w4ec_stack_forward(s, _ptr(x), _ptr(y), M, flags, _stream(stream)), "spear_w4ec_stack_forward")
+
+
+def spear_w4ec_stack_forward_host(s: int, x_host, y_host, M: int, flags: int = 0, stream=None):
+    _check(_lib.spear_w4ec_stack_forward_host(s, _ptr(x_host), _ptr(y_host), M, flags, _stream(stream)),
+           "spear_w4ec_stack_forward_host")
+
+
+def spear_w4ec_stack_buffer(s: int, index: int) -> int:
+    p = ctypes.c_void_p()
+    _check(_lib.spear_w4ec_stack_buffer(s, index, ctypes.byref(p)), "spear_w4ec_stack_buffer")
+    return p.value
+
+
+def spear_w4ec_stack_destroy(s: int):
+    _check(_lib.spear_w4ec_stack_destroy(s), "spear_w4ec_stack_destroy")
+
+
 class W4ECLinear:
     """Owning wrapper of one packed layer (create + pack; destroy on close).
 
@@ -234,6 +274,70 @@ class W4ECLinear:
     def close(self):
         if getattr(self, "h", None):
             spear_w4ec_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class W4ECStack:
+    """Owning wrapper of a layer stack (spear_w4ec_stack_*).
+
+    ops: sequence of (W4ECLinear, in, out, ec): buffer 0 is the input x,
+    1 the output y (last op only), 2 and up intermediates; ec = 1 places the
+    layer's EC, 0 runs it as the plain W4 GEMM.  The layers must stay open
+    while the stack is used.
+    """
+
+    def __init__(self, ops, max_M: int):
+        self.layers = [op[0] for op in ops]
+        readers = [op[0].K for op in ops if op[1] == 0]
+        self.in_width = readers[0] if readers else 0   # the library rejects a stack that never reads x
+        self.out_width = ops[-1][0].N
+        self.max_M = max_M
+        self.device = ops[0][0].device
+        self.h = spear_w4ec_stack_create([(lin.h, i, o, e) for (lin, i, o, e) in ops], max_M)
+        self.widths = {}
+        for lin, _, o, _ in ops:
+            self.widths[o] = lin.N
+
+    def forward(self, x: torch.Tensor, flags: int = 0, out: torch.Tensor | None = None, stream=None):
+        M = x.shape[0]
+        _dev_bf16(x, (M, self.in_width), "x")
+        y = out if out is not None else torch.empty((M, self.out_width), dtype=torch.bfloat16, device=x.device)
+        _dev_bf16(y, (M, self.out_width), "y")
+        spear_w4ec_stack_forward(self.h, x, y, M, flags, stream)
+        return y
+
+    __call__ = forward
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, flags: int = 0, stream=None):
+        M = x_host.shape[0]
+        if x_host.is_cuda or y_host.is_cuda or tuple(x_host.shape) != (M, self.in_width) or \
+                tuple(y_host.shape) != (M, self.out_width) or x_host.dtype != torch.bfloat16 or \
+                y_host.dtype != torch.bfloat16 or not (x_host.is_contiguous() and y_host.is_contiguous()):
+            raise ValueError("x_host, y_host must be contiguous host bf16 tensors [M, in] and [M, out]")
+        spear_w4ec_stack_forward_host(self.h, x_host, y_host, M, flags, stream)
+        return y_host
+
+    def buffer(self, index: int, M: int) -> torch.Tensor:
+        """A copy of intermediate buffer ``index`` as written by the last forward on M tokens."""
+        ptr = spear_w4ec_stack_buffer(self.h, index)
+        width = self.widths[index]
+
+        class _View:   # the buffer's first M rows, seen through the CUDA array interface
+            __cuda_array_interface__ = {"shape": (M, width), "typestr": "<i2", "data": (ptr, False),
+                                        "version": 2, "strides": None}
+
+        torch.cuda.synchronize(self.device)
+        return torch.as_tensor(_View(), device=self.device).view(torch.bfloat16).clone()
+
+    def close(self):
+        if getattr(self, "h", None):
+            spear_w4ec_stack_destroy(self.h)
             self.h = None
 
     def __del__(self):
