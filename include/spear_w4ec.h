@@ -98,6 +98,33 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r,
 int spear_w4ec_pack(spear_w4ec *h, const void *W, const void *A, const void *B,
                     const void *w_g, float b_g, void *stream);
 
+/* The same as spear_w4ec_pack with the asymmetric (min-max) per-channel
+ * rule and a stored zero point, the form that the abstract's "state-of-the-art
+ * 4-bit quantizers" commonly use per channel (the pages give no rule; this is
+ * the library's reading):
+ *   lo = min(0, min_k W[n,k]),  hi = max(0, max_k W[n,k])
+ *   s[n] = fp32(fp32(hi - lo) / 15)
+ *   z[n] = clamp(round_half_even(fp32(-lo / s[n])), 0, 15)
+ *   q    = clamp(round_half_even(fp32(W[n,k] / s[n])) + z[n], 0, 15)
+ *   an all-zero row has s = 0, z = 8 and every code 8.
+ * Codes, scales and zero points are bit-identical to this definition. */
+int spear_w4ec_pack_asym(spear_w4ec *h, const void *W, const void *A, const void *B,
+                         const void *w_g, float b_g, void *stream);
+
+/* Import a layer quantised by any per-channel 4-bit quantiser (SPEAR,
+ * Abstract: the Error Compensators sit on top of existing 4-bit quantizers):
+ *   codes dev uint32 [N][K/8]  the exported layout (code of k = 8j+i in bits
+ *                              [4i, 4i+3] of word j of row n)
+ *   s     dev float [N]        per-channel scale
+ *   z     dev uint8 [N]        per-channel zero point, 0..15
+ * so that w^[n,k] = s[n] * (q[n,k] - z[n]); A, B, w_g and b_g as in
+ * spear_w4ec_pack.  spear_w4ec_get_packed returns the three arrays bit for
+ * bit.  A zero point above 15 or a non-finite scale is reported as
+ * SPEAR_ERR_DEVICE by spear_w4ec_sync_status.  The inputs may be freed once
+ * the stream work of this call has completed. */
+int spear_w4ec_import(spear_w4ec *h, const void *codes, const float *s, const uint8_t *z,
+                      const void *A, const void *B, const void *w_g, float b_g, void *stream);
+
 /* y = x.W^T + g.(x.A).B for M tokens.
  *   x  dev bf16 [M][K], 16-byte aligned;  y  dev bf16 [M][N], 16-byte aligned.
  * 0 <= M <= max_M (M = 0 is a no-op).  flags: SPEAR_* above (0 = dispatch).

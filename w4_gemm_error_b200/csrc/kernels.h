@@ -37,9 +37,14 @@ struct Packed {
     float b_g;
 };
 
-// ---- pack: per-channel RTN int4 of W, plus the EC operand layouts
+// ---- pack: per-channel RTN int4 of W (symmetric, z = 8, or asymmetric
+// min-max with a stored zero point), plus the EC operand layouts
 cudaError_t launch_pack(const Packed &pk, const void *W, const void *A, const void *B,
-                        const void *wg, int *status, cudaStream_t st);
+                        const void *wg, int *status, cudaStream_t st, bool asym);
+// codes quantised elsewhere ([N][K/8], exported nibble order), s [N], z [N]
+// into the device layout, plus the EC operand layouts
+cudaError_t launch_import(const Packed &pk, const void *codes, const float *s, const uint8_t *z, const void *A,
+                          const void *B, const void *wg, int *status, cudaStream_t st);
 // codes in the exported layout [N][K/8] (row-major, no padding)
 cudaError_t launch_untile_codes(const Packed &pk, uint32_t *dst, cudaStream_t st);
 

@@ -191,6 +191,33 @@ int run_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t
     return SPEAR_OK;
 }
 
+// Pack (W given: symmetric or asymmetric RTN) or import (codes, s, z given)
+// the layer, then the EC operands and the kernels' tensor maps.
+int pack_layer(spear_w4ec *h, const void *W, const void *codes, const float *s, const uint8_t *z, const void *A,
+               const void *B, const void *w_g, float b_g, void *stream, bool asym)
+{
+    if (!h || (W && !aligned16(W)) || (!W && !codes))
+        return SPEAR_ERR_INVALID;
+    if (h->pk.r > 0 && (!A || !B || !w_g))
+        return SPEAR_ERR_INVALID;
+    DeviceGuard guard(h->device);
+    if (!guard.ok())
+        return SPEAR_ERR_CUDA;
+    h->pk.b_g = b_g;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = W ? launch_pack(h->pk, W, A, B, w_g, h->status, st, asym)
+                      : launch_import(h->pk, codes, s, z, A, B, w_g, h->status, st);
+    if (e != cudaSuccess)
+        return from_cuda(e);
+    e = tc_prepare(h->pk, h->tc);
+    if (e == cudaSuccess)
+        e = decode_prepare(h->pk, h->dec);
+    if (e != cudaSuccess)
+        return from_cuda(e);
+    h->packed = true;
+    return SPEAR_OK;
+}
+
 }  // namespace
 
 namespace spear {
@@ -297,24 +324,21 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r, const s
 int spear_w4ec_pack(spear_w4ec *h, const void *W, const void *A, const void *B, const void *w_g, float b_g,
                     void *stream)
 {
-    if (!h || !W || !aligned16(W))
+    return pack_layer(h, W, nullptr, nullptr, nullptr, A, B, w_g, b_g, stream, false);
+}
+
+int spear_w4ec_pack_asym(spear_w4ec *h, const void *W, const void *A, const void *B, const void *w_g, float b_g,
+                         void *stream)
+{
+    return pack_layer(h, W, nullptr, nullptr, nullptr, A, B, w_g, b_g, stream, true);
+}
+
+int spear_w4ec_import(spear_w4ec *h, const void *codes, const float *s, const uint8_t *z, const void *A,
+                      const void *B, const void *w_g, float b_g, void *stream)
+{
+    if (!codes || !s || !z)
         return SPEAR_ERR_INVALID;
-    if (h->pk.r > 0 && (!A || !B || !w_g))
-        return SPEAR_ERR_INVALID;
-    DeviceGuard guard(h->device);
-    if (!guard.ok())
-        return SPEAR_ERR_CUDA;
-    h->pk.b_g = b_g;
-    cudaError_t e = launch_pack(h->pk, W, A, B, w_g, h->status, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess)
-        return from_cuda(e);
-    e = tc_prepare(h->pk, h->tc);
-    if (e == cudaSuccess)
-        e = decode_prepare(h->pk, h->dec);
-    if (e != cudaSuccess)
-        return from_cuda(e);
-    h->packed = true;
-    return SPEAR_OK;
+    return pack_layer(h, nullptr, codes, s, z, A, B, w_g, b_g, stream, false);
 }
 
 int spear_w4ec_forward(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t flags, void *stream)

@@ -30,7 +30,8 @@ SPEAR_FORCE_SPLIT = 4
 SPEAR_FORCE_DECODE = 8
 SPEAR_FORCE_TC = 16
 
-EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_forward", "spear_w4ec_forward_host",
+EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_pack_asym", "spear_w4ec_import",
+            "spear_w4ec_forward", "spear_w4ec_forward_host",
             "spear_w4ec_destroy", "spear_w4ec_get_packed", "spear_w4ec_get_gate", "spear_w4ec_sync_status",
             "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_gate_noalloc", "spear_w4ec_set_next",
             "spear_w4ec_stack_create", "spear_w4ec_stack_forward", "spear_w4ec_stack_forward_host",
@@ -62,6 +63,8 @@ def _load():
     sig = {
         "spear_w4ec_create": [ctypes.POINTER(P), i64, i64, i32, ctypes.POINTER(_Opts)],
         "spear_w4ec_pack": [P, P, P, P, P, f32, P],
+        "spear_w4ec_pack_asym": [P, P, P, P, P, f32, P],
+        "spear_w4ec_import": [P, P, P, P, P, P, P, f32, P],
         "spear_w4ec_forward": [P, P, P, i64, u32, P],
         "spear_w4ec_forward_host": [P, P, P, i64, u32, P],
         "spear_w4ec_destroy": [P],
@@ -132,6 +135,16 @@ def spear_w4ec_create(K: int, N: int, r: int, max_M: int = 4096, device: int = -
 def spear_w4ec_pack(h: int, W, A, B, w_g, b_g: float, stream=None):
     _check(_lib.spear_w4ec_pack(h, _ptr(W), _ptr(A), _ptr(B), _ptr(w_g), float(b_g), _stream(stream)),
            "spear_w4ec_pack")
+
+
+def spear_w4ec_pack_asym(h: int, W, A, B, w_g, b_g: float, stream=None):
+    _check(_lib.spear_w4ec_pack_asym(h, _ptr(W), _ptr(A), _ptr(B), _ptr(w_g), float(b_g), _stream(stream)),
+           "spear_w4ec_pack_asym")
+
+
+def spear_w4ec_import(h: int, codes, s, z, A, B, w_g, b_g: float, stream=None):
+    _check(_lib.spear_w4ec_import(h, _ptr(codes), _ptr(s), _ptr(z), _ptr(A), _ptr(B), _ptr(w_g), float(b_g),
+                                  _stream(stream)), "spear_w4ec_import")
 
 
 def spear_w4ec_forward(h: int, x, y, M: int, flags: int = 0, stream=None):
@@ -214,20 +227,41 @@ class W4ECLinear:
     Shapes: W [N, K], A [K, r], B [r, N], w_g [K] (bf16 CUDA tensors).
     """
 
-    def __init__(self, W: torch.Tensor, A: torch.Tensor | None, B: torch.Tensor | None,
-                 w_g: torch.Tensor | None, b_g: float, max_M: int = 4096, stream=None):
-        N, K = W.shape
+    def __init__(self, W: torch.Tensor | None, A: torch.Tensor | None, B: torch.Tensor | None,
+                 w_g: torch.Tensor | None, b_g: float, max_M: int = 4096, stream=None, quant: str = "sym",
+                 packed=None):
+        """quant: "sym" (spear_w4ec_pack) or "asym" (spear_w4ec_pack_asym);
+        packed: (codes int32/uint32 [N, K/8], s float32 [N], z uint8 [N]) CUDA
+        tensors of a layer quantised elsewhere (spear_w4ec_import; W is None)."""
+        if packed is not None:
+            codes, s_, z_ = packed
+            N, K = codes.shape[0], codes.shape[1] * 8
+            if not (codes.is_cuda and codes.dtype in (torch.int32, torch.uint32) and codes.is_contiguous()
+                    and s_.is_cuda and s_.dtype == torch.float32 and tuple(s_.shape) == (N,)
+                    and z_.is_cuda and z_.dtype == torch.uint8 and tuple(z_.shape) == (N,)):
+                raise ValueError("packed must be CUDA (codes [N, K/8] int32, s [N] float32, z [N] uint8)")
+            device = codes.device
+        else:
+            N, K = W.shape
+            _dev_bf16(W, (N, K), "W")
+            device = W.device
+        if quant not in ("sym", "asym"):
+            raise ValueError("quant must be 'sym' or 'asym'")
         r = 0 if A is None else A.shape[1]
-        _dev_bf16(W, (N, K), "W")
         if r:
             _dev_bf16(A, (K, r), "A")
             _dev_bf16(B, (r, N), "B")
             _dev_bf16(w_g, (K,), "w_g")
         self.K, self.N, self.r, self.max_M = K, N, r, max_M
-        self.device = W.device
-        self.h = spear_w4ec_create(K, N, r, max_M, W.device.index if W.device.index is not None else -1)
+        self.device = device
+        self.h = spear_w4ec_create(K, N, r, max_M, device.index if device.index is not None else -1)
         try:
-            spear_w4ec_pack(self.h, W, A, B, w_g, b_g, stream)
+            if packed is not None:
+                spear_w4ec_import(self.h, packed[0], packed[1], packed[2], A, B, w_g, b_g, stream)
+            elif quant == "asym":
+                spear_w4ec_pack_asym(self.h, W, A, B, w_g, b_g, stream)
+            else:
+                spear_w4ec_pack(self.h, W, A, B, w_g, b_g, stream)
         except Exception:
             spear_w4ec_destroy(self.h)
             self.h = None
