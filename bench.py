@@ -231,15 +231,6 @@ def measure_workload(name, args, rank, world, local_rank, cpu_seconds):
             layers.append(spear.W4ECLinear(W, A, B, wg, base.b_g, max_M=max(Ms), stream=stream))
         del W0, A0, B0
     torch.cuda.synchronize(dev)
-    if args.tune:
-        # the library's adaptive dispatch: each layer times its legal paths once per batch size
-        xs_t = {M: make_x(M, K, seed=0).to(dev) for M in Ms}
-        y_t = {M: torch.empty((M, N), dtype=torch.bfloat16, device=dev) for M in Ms}
-        with torch.cuda.stream(stream):
-            for M in Ms:
-                for lin in layers:
-                    lin.tune(xs_t[M], y_t[M], stream=stream)
-        torch.cuda.synchronize(dev)
     # the step's layer sequence as one stack (spear_w4ec_stack_*): chained
     # (square layers: y of layer l is x of layer l + 1) or all reading x;
     # intermediates alternate between two buffers; every EC placed
@@ -294,11 +285,45 @@ def measure_workload(name, args, rank, world, local_rank, cpu_seconds):
             dist.barrier()
         return ms, (sampler.summary() if sampler else None)
 
-    g_on = capture(0)
-    g_off = capture(spear.SPEAR_EC_OFF)
-    ms_on, clocks = timed(g_on, args.steps, args.warmup, sample_clocks=True)
+    # the library's default dispatch, then the adaptive one: layer 0 times every
+    # legal path per batch size (spear_w4ec_tune), its table goes out as JSON and
+    # into every layer (spear_w4ec_table_save / _load; the layers share a shape);
+    # the faster of the two is the step that is reported
+    g_def_on, g_def_off = capture(0), capture(spear.SPEAR_EC_OFF)
+    paths_default = {str(M): path_name(layers[0].dispatch(M)) for M in Ms}
+    table_text = None
+    if not args.no_tune:
+        with torch.cuda.stream(stream):
+            for M in Ms:
+                layers[0].tune(xs[M], ys[M], stream=stream)
+        torch.cuda.synchronize(dev)
+        table_text = layers[0].table_json()
+        for lin in layers[1:]:
+            lin.load_table(table_text)
+    paths_tuned = {str(M): path_name(layers[0].dispatch(M)) for M in Ms}
+    ms_def, clocks_def = timed(g_def_on, args.steps, args.warmup, sample_clocks=True)
+    if table_text is not None and paths_tuned != paths_default:
+        g_tun_on, g_tun_off = capture(0), capture(spear.SPEAR_EC_OFF)
+        ms_tun, clocks_tun = timed(g_tun_on, args.steps, args.warmup, sample_clocks=True)
+    else:
+        g_tun_on = g_tun_off = None
+        ms_tun, clocks_tun = float("inf"), None
+    tuned_wins = ms_tun < ms_def
+    if tuned_wins:
+        ms_on, clocks, g_off = ms_tun, clocks_tun, g_tun_off
+        paths = paths_tuned
+    else:
+        ms_on, clocks, g_off = ms_def, clocks_def, g_def_off
+        paths = paths_default
+        if table_text is not None:
+            # back to the default rule for the end-to-end run below
+            untuned = json.loads(table_text)
+            for b in untuned["buckets"]:
+                b["choice"] = None
+            for lin in layers:
+                lin.load_table(json.dumps(untuned))
     ms_off, _ = timed(g_off, args.steps, args.warmup)
-    del g_on, g_off
+    del g_def_on, g_def_off, g_tun_on, g_tun_off
 
     forwards_per_step = L * len(Ms)
     if wl["kind"] == "decode":
@@ -357,7 +382,7 @@ def measure_workload(name, args, rank, world, local_rank, cpu_seconds):
 
     launches_per_forward = {}
     for M in Ms:
-        ch = layers[0].dispatch(M)
+        ch = layers[0].dispatch(M)   # the dispatch of the reported step
         if ch & spear.SPEAR_FORCE_DECODE:
             split = bool(r and ch & spear.SPEAR_FORCE_SPLIT)
             n = math.ceil(M / 32) + (2 if split else 0)   # split: prepass + separate EC kernel
@@ -383,8 +408,13 @@ def measure_workload(name, args, rank, world, local_rank, cpu_seconds):
                        "graph": "one CUDA graph per step, kernels chained with programmatic dependent launch",
                        "prefetch": "off" if args.no_prefetch else
                                    "each layer's decode kernel reads the next layer's codes from HBM into L2",
-                       "dispatch": "tuned (spear_w4ec_tune per layer and M)" if args.tune else "library default",
-                       "paths": {str(M): path_name(layers[0].dispatch(M)) for M in Ms},
+                       "dispatch": ("tuned (spear_w4ec_tune on layer 0 per M, table loaded into every layer as "
+                                    "JSON): faster than the default rule") if tuned_wins else
+                                   ("library default rule" + ("" if table_text is None else
+                                    " (the tuned table was measured too and was not faster)")),
+                       "paths": paths,
+                       "step_ms": {"default": round(ms_def / args.steps, 4),
+                                   "tuned": None if ms_tun == float("inf") else round(ms_tun / args.steps, 4)},
                        "parallelism": f"replicas x{world}"},
             "ec_overhead": round(ec_overhead, 4),
             "e2e": {"value": round(e2e_value, 2), "unit": unit, "h2d_bytes_per_step": h2d,
@@ -539,9 +569,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefetch", action="store_true",
                     help="do not chain the layers with the cross-layer L2 prefetch hint")
-    ap.add_argument("--tune", action="store_true",
-                    help="time every path per layer and M first (spear_w4ec_tune); the default dispatch is the "
-                         "library's rule, which a profiler cannot perturb")
+    ap.add_argument("--no-tune", action="store_true",
+                    help="skip the adaptive dispatch (spear_w4ec_tune) and report the library's default rule")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

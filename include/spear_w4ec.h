@@ -171,6 +171,39 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
  * tiles fill at most half of the SMs). */
 int spear_w4ec_dispatch(const spear_w4ec *h, int64_t M, uint32_t *choice);
 
+/* Cost model for an EC-aware scheduler (SPEAR, Abstract: an SLO-constrained
+ * EC-aware scheduler keeps serving predictable; the scheduler itself is not
+ * part of this library).  After spear_w4ec_tune has run for M's bucket, *us
+ * receives the measured median time in microseconds of one forward with
+ *   flags = SPEAR_FORCE_DECODE or SPEAR_FORCE_TC,
+ *         | SPEAR_FORCE_FUSED or SPEAR_FORCE_SPLIT (EC placement),
+ *         | SPEAR_EC_OFF optionally (the same path without the EC; the
+ *           placement flag is then ignored),
+ * so that a scheduler can weigh the EC's price per batch size.  Returns
+ * SPEAR_ERR_STATE if that choice was not measured (not tuned, or the path
+ * cannot run this layer), SPEAR_ERR_INVALID for flags that name no single
+ * choice.  Host-only; no device work. */
+int spear_w4ec_cost(const spear_w4ec *h, int64_t M, uint32_t flags, float *us);
+
+/* Save the handle's dispatch table (the tuned choice and measured costs of
+ * every bucket tuned so far) as JSON text into buf (cap bytes, including the
+ * terminating NUL); *len receives the text's length without the NUL.  If buf
+ * is NULL or too small, returns SPEAR_ERR_INVALID with *len set, so a caller
+ * can size the buffer and call again.  Host-only.  The text records K, N and r
+ * and, per bucket: {"bucket": b, "M_max": 2^b (-1 for the last), "choice":
+ * "decode+fused" | "decode+split" | "tcgen05+fused" | "tcgen05+split" | null,
+ * "us": {name: microseconds, ...}}. */
+int spear_w4ec_table_save(const spear_w4ec *h, char *buf, size_t cap, size_t *len);
+
+/* Load a table saved by spear_w4ec_table_save (NUL-terminated JSON) into a
+ * handle of the same K, N and r, replacing the buckets it lists; forward then
+ * follows the loaded choices as if spear_w4ec_tune had chosen them.
+ * SPEAR_ERR_INVALID for text that does not parse, another layer shape or a
+ * malformed entry; SPEAR_ERR_UNSUPPORTED for a choice whose path cannot run
+ * this layer on this device.  Nothing changes unless the whole table is
+ * accepted.  Host-only. */
+int spear_w4ec_table_load(spear_w4ec *h, const char *json);
+
 /* Cross-layer weight prefetch, a hint for serving loops that run a fixed
  * sequence of layers (the SPEAR pages do not describe one).  `next` names the
  * layer whose forward follows h's forward on the same stream (h itself is

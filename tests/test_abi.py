@@ -88,3 +88,14 @@ def test_stack_calls_reject_bad_arguments_before_touching_the_device(lib):
     p = ctypes.c_void_p()
     assert L.spear_w4ec_stack_buffer(None, 2, ctypes.byref(p)) == spear.SPEAR_ERR_INVALID
     assert L.spear_w4ec_stack_destroy(None) == spear.SPEAR_OK
+
+
+def test_table_and_cost_calls_reject_bad_arguments_before_touching_the_device(lib):
+    from w4_gemm_error_b200 import spear
+    L = spear.lib()
+    n = ctypes.c_size_t(7)
+    us = ctypes.c_float(0)
+    assert L.spear_w4ec_table_save(None, None, 0, ctypes.byref(n)) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_table_load(None, b"{}") == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_cost(None, 1, spear.SPEAR_FORCE_DECODE | spear.SPEAR_FORCE_FUSED, ctypes.byref(us)) \
+        == spear.SPEAR_ERR_INVALID

@@ -74,6 +74,28 @@ def test_decode_mlp_larger_batches_sampled(M, K, N):
     P.close()
 
 
+# Decode kernel with K split over a cluster (up to 16 tokens, K >= 512):
+# shapes chosen to reach its corners.  1032 x 264: K split in two with an odd
+# chunk count (the ranks hold 3 and 2 chunks, one stage of a single chunk);
+# 14336 x 4096: eight-way split with 7 chunks per rank and two EC units per
+# CTA (both G buffers cycle); 2048 x 8192: four groups of tiles per cluster;
+# 4096 x 1000: ragged rows, two token groups; 8192 x 2048 without an EC;
+# 4096 x 14336 at rank 128: nine 16-row groups of G (the most it takes).
+@pytest.mark.parametrize("M,K,N,r", [(5, 1032, 264, 20), (16, 14336, 4096, 64), (3, 2048, 8192, 32),
+                                     (12, 4096, 1000, 48), (1, 8192, 2048, 0), (9, 4096, 14336, 128)])
+def test_cluster_split_decode_shapes(M, K, N, r, monkeypatch):
+    monkeypatch.setenv("SPEAR_DECODE_STREAM", "1")
+    P = Problem(M, K, N, r, seed=M + K + N)
+    ref = P.oracle_y()
+    flag_sets = (DECODE | FUSED, DECODE | SPLIT) if r else (DECODE | FUSED,)
+    for flags in flag_sets:
+        assert_close(_run(P, flags), ref, f"flags={flags}")
+    assert_close(_run(P, DECODE | EC_OFF), P.oracle_y(ec_on=False), "EC off")
+    y1 = _run(P, DECODE | FUSED)
+    assert torch.equal(_run(P, DECODE | FUSED), y1), "repeated runs differ"
+    P.close()
+
+
 def test_ec_isolated_on_qo_shape():
     """y(EC on) - y(EC off) against the oracle's correction term alone."""
     P = Problem(16, 4096, 4096, 32, seed=3)

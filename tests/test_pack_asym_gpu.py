@@ -71,11 +71,23 @@ def test_pack_asym_golden_and_edge_rows():
         if line and line[0].startswith("row"):
             rows.append([float(v) for v in line[1:]])
     W = np.array(rows)
-    tiny = np.full((1, 16), 2.0 ** -130)
+    tiny = np.full((1, 16), 2.0 ** -130)            # subnormal range: no flush to zero
     tiny[0, 3] = -(2.0 ** -129)
-    pos = np.abs(np.random.default_rng(1).standard_normal((1, 16)))
-    neg = -pos
-    _check(to_bf16(np.concatenate([W, tiny, pos, neg, np.zeros((1, 16))])))
+    rng = np.random.default_rng(1)
+    pos = np.abs(rng.standard_normal((2, 16)))       # all-positive and all-negative rows
+    neg = -np.abs(rng.standard_normal((2, 16)))
+    one = np.zeros((1, 16))
+    one[0, 9] = -3.0                                  # a single nonzero weight
+    const = np.full((1, 16), 0.75)                    # a constant row
+    huge = np.full((1, 16), 3.0e38)                    # range near the top of fp32
+    huge[0, 5] = -1.0
+    ztie = np.linspace(-0.3125, 1.5625, 16)[None, :]  # -lo / s = 2.5: the zero point ties to 2
+    ztie = np.round(ztie * 64) / 64
+    ztie[0, 0], ztie[0, -1] = -0.3125, 1.5625
+    alt = np.tile([0.5, -0.5], 8)[None, :]
+    rows = np.concatenate([W, tiny, pos, neg, one, const, huge, ztie, alt, np.zeros((1, 16))])
+    assert rows.shape[0] % 8 == 0                     # N must be a multiple of 8
+    _check(to_bf16(rows))
 
 
 def test_import_keeps_codes_scales_and_zero_points():

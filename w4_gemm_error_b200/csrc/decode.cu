@@ -45,6 +45,7 @@
 //    with a bounded wait (about a second) that records a timeout in the
 //    handle's status word instead of hanging.
 #include <algorithm>
+#include <cstdlib>
 #include <new>
 
 #include "async_utils.cuh"
@@ -70,6 +71,7 @@ struct Maps {
     CUtensorMap bt;       // [Np][rp] bf16, boxes of rp x 64
     int g3;               // g is the 3-D view (else 2-D boxes of 64 k x 16 rows)
     void *rows;           // maps of the row-CTA kernel (decode_rows.cu), null if it does not fit
+    void *stream;         // maps of the cluster-split kernel (decode_stream.cu), null if it does not fit
 };
 
 struct DecodeParams {
@@ -716,6 +718,14 @@ const void *kernel_ptr()
 
 }  // namespace
 
+// The cluster-split decode kernel (decode_stream.cu) serves up to 16 tokens
+// when SPEAR_DECODE_STREAM=1; otherwise the row-CTA and split-K kernels do.
+bool decode_stream_enabled()
+{
+    const char *v = std::getenv("SPEAR_DECODE_STREAM");
+    return v && v[0] == '1';
+}
+
 bool decode_supported(const Packed &pk, int num_sms)
 {
     if (pk.rp > 128)
@@ -768,13 +778,17 @@ cudaError_t decode_prepare(const Packed &pk, DecodeWork &w)
     }
     if (e == cudaSuccess && decode_rows_shape(pk))
         e = decode_rows_prepare(pk, &m->rows);
+    if (e == cudaSuccess && decode_stream_shape(pk))
+        e = decode_stream_prepare(pk, &m->stream);
     return e;
 }
 
 void decode_free(DecodeWork &w)
 {
-    if (w.maps)
+    if (w.maps) {
         decode_rows_free(static_cast<Maps *>(w.maps)->rows);
+        decode_stream_free(static_cast<Maps *>(w.maps)->stream);
+    }
     delete static_cast<Maps *>(w.maps);
     w.maps = nullptr;
 }
@@ -790,6 +804,9 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     if (M > kDecodeMaxTokens || !w.maps)
         return cudaErrorInvalidValue;
     const Maps *m = static_cast<const Maps *>(w.maps);
+    // up to 16 tokens: K split over a cluster, each CTA with its slice of x
+    if (m->stream && decode_stream_enabled() && decode_stream_fits(pk, M, num_sms))
+        return launch_decode_stream(pk, m->stream, x, y, M, ec, w, status, st, num_sms);
     // up to 16 tokens on a layer whose 16-row slices fit in shared memory: one
     // CTA per 16 rows over the whole of K, no exchange between CTAs
     if (m->rows && decode_rows_fits(pk, M, num_sms))

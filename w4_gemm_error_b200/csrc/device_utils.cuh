@@ -49,6 +49,16 @@ __device__ __forceinline__ uint32_t dequant_pair(uint32_t w_shifted, uint32_t ne
     return fma_bf16x2(t, 0x3F803F80u /* (1.0, 1.0) */, neg_bias);
 }
 
+// As dequant_pair with a per-row multiplier: mul = bf16x2(1, 1) with neg_bias
+// as above, or mul = neg_bias = 0 for a row whose scale is 0 (its weights are
+// 0 whatever its codes say), for a kernel that applies a stand-in scale of 1
+// to such rows after accumulating.
+__device__ __forceinline__ uint32_t dequant_pair_mul(uint32_t w_shifted, uint32_t mul, uint32_t neg_bias)
+{
+    const uint32_t t = lop3_and_or(w_shifted, 0x000F000Fu, 0x43004300u);
+    return fma_bf16x2(t, mul, neg_bias);
+}
+
 // D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col).  Not volatile: its
 // only effect is on d, so the compiler may interleave independent MMAs.
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,

@@ -35,6 +35,9 @@ struct spear_w4ec {
     void *y_stage = nullptr;
     // dispatch table: flags per M bucket, 0 = not tuned
     uint32_t table[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+    // measured microseconds per forward, per M bucket and choice (see
+    // spear::cost_index), negative where not measured
+    float cost_us[9][8];
     // host-side fault injection (SPEAR_FAULT=alloc|launch|timeout)
     bool fault_launch = false;
     bool fault_timeout = false;
@@ -72,6 +75,21 @@ class DeviceGuard {
 
 // Status of a CUDA runtime result (SPEAR_ERR_NOMEM for an allocation failure).
 int status_of(cudaError_t e);
+
+// Slot of a (path, EC placement, EC on/off) choice in cost_us: tcgen05 path
+// + 4, split EC + 2, EC off + 1 (EC off ignores the placement; its time is
+// kept in both placement slots).
+inline int cost_index(uint32_t flags)
+{
+    return ((flags & SPEAR_FORCE_TC) ? 4 : 0) + ((flags & SPEAR_FORCE_SPLIT) ? 2 : 0) + ((flags & SPEAR_EC_OFF) ? 1 : 0);
+}
+
+// M bucket of the dispatch table: 1, 2, 4, ..., 128 -> 0..7, more -> 8.
+int bucket_of(int64_t M);
+
+// Whether the handle's device can run a kernel family (SPEAR_FORCE_DECODE or
+// SPEAR_FORCE_TC) on this layer.
+bool path_supported(const spear_w4ec *h, uint32_t path);
 
 // The kernel sequence of one forward pass of a packed layer.  The caller has
 // checked the arguments (1 <= M <= max_M, 16-byte aligned device x and y) and

@@ -80,6 +80,11 @@ struct DecodeWork {
     // kernels once their own codes have landed), null for none
     const void *pf;
     size_t pf_bytes;
+    // cluster-split decode kernel (decode_stream.cu): partials of the EC
+    // down-projection and u (decode_stream_ws_floats), and its counters
+    // (kDecodeStreamCounters, zero between calls)
+    float *ws_stream;
+    unsigned *cnt_stream;
 };
 constexpr int kDecodeMaxTokens = 32;   // tokens per launch
 bool decode_supported(const Packed &pk, int num_sms);
@@ -99,6 +104,19 @@ cudaError_t decode_rows_prepare(const Packed &pk, void **maps);
 void decode_rows_free(void *maps);
 cudaError_t launch_decode_rows(const Packed &pk, const void *maps, const void *x, void *y, int64_t M, bool ec,
                                const DecodeWork &w, int *status, cudaStream_t st, int num_sms);
+
+// ---- decode kernel for up to 16 tokens with K split over a thread-block
+// cluster (each CTA stages only its slice of x; partial tiles summed over
+// distributed shared memory; EC down-projection in small units with a
+// last-arriver reduction).  launch_decode takes it when it fits.
+constexpr int kDecodeStreamCounters = 2 + 9;
+bool decode_stream_shape(const Packed &pk);
+bool decode_stream_fits(const Packed &pk, int64_t M, int num_sms);
+size_t decode_stream_ws_floats(const Packed &pk);
+cudaError_t decode_stream_prepare(const Packed &pk, void **maps);
+void decode_stream_free(void *maps);
+cudaError_t launch_decode_stream(const Packed &pk, const void *maps, const void *x, void *y, int64_t M, bool ec,
+                                 const DecodeWork &w, int *status, cudaStream_t st, int num_sms);
 
 // ---- split EC: y[t][n] = bf16(y[t][n] + sum_j v[t][j] * Bt[n][j]), v in fp32
 cudaError_t launch_ec_apply(const Packed &pk, const float *vf, void *y, int64_t M, cudaStream_t st);

@@ -32,17 +32,6 @@ int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int bucket_of(int64_t M)
-{
-    int b = 0;
-    int64_t cap = 1;
-    while (b < 8 && M > cap) {
-        cap *= 2;
-        ++b;
-    }
-    return b;  // 1,2,4,...,128 -> 0..7, >128 -> 8
-}
-
 template <class T>
 cudaError_t alloc_zero(T **p, size_t count)
 {
@@ -69,6 +58,8 @@ void free_all(spear_w4ec *h)
     cudaFree(h->pre.counters);
     cudaFree(h->dec.ws_u);
     cudaFree(h->dec.flags);
+    cudaFree(h->dec.ws_stream);
+    cudaFree(h->dec.cnt_stream);
     decode_free(h->dec);
     tc_free(h->tc);
     cudaFree(h->status);
@@ -224,6 +215,26 @@ namespace spear {
 
 int status_of(cudaError_t e) { return from_cuda(e); }
 
+int bucket_of(int64_t M)
+{
+    int b = 0;
+    int64_t cap = 1;
+    while (b < 8 && M > cap) {
+        cap *= 2;
+        ++b;
+    }
+    return b;  // 1,2,4,...,128 -> 0..7, >128 -> 8
+}
+
+bool path_supported(const spear_w4ec *h, uint32_t path)
+{
+    if (path == SPEAR_FORCE_TC)
+        return tc_supported(h);
+    if (path == SPEAR_FORCE_DECODE)
+        return decode_supported(h->pk, h->num_sms);
+    return false;
+}
+
 int forward_checked(const spear_w4ec *h, const void *x, void *y, int64_t M, uint32_t flags, cudaStream_t st)
 {
     return run_forward(h, x, y, M, flags, st);
@@ -273,6 +284,9 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r, const s
     h->device = dev;
     h->max_M = (opts && opts->max_M > 0) ? opts->max_M : 4096;
     cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, dev);
+    for (auto &row : h->cost_us)
+        for (float &c : row)
+            c = -1.0f;
     h->fault_launch = std::strcmp(env_fault(), "launch") == 0;
     h->fault_timeout = std::strcmp(env_fault(), "timeout") == 0;
 
@@ -307,6 +321,8 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r, const s
     }
     chk(alloc_zero(&h->dec.ws_u, decode_u_floats(pk)));
     chk(alloc_zero(&h->dec.flags, (size_t)2));
+    chk(alloc_zero(&h->dec.ws_stream, decode_stream_ws_floats(pk)));
+    chk(alloc_zero(&h->dec.cnt_stream, (size_t)kDecodeStreamCounters));
     chk(tc_alloc(pk, h->max_M, h->num_sms, h->tc));
     chk(alloc_zero(&h->status, 1));
     chk(alloc_zero(&h->vready, 2));
@@ -515,16 +531,17 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
         return SPEAR_ERR_INVALID;
     DeviceGuard guard(h->device);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // every legal choice with the EC (fused and split), and each path with the EC off
     std::vector<uint32_t> cands;
     const uint32_t paths[2] = {SPEAR_FORCE_DECODE, SPEAR_FORCE_TC};
     for (uint32_t path : paths) {
-        if (path == SPEAR_FORCE_TC && !tc_supported(h))
-            continue;
-        if (path == SPEAR_FORCE_DECODE && !decode_supported(h->pk, h->num_sms))
+        if (!path_supported(h, path))
             continue;
         cands.push_back(path | SPEAR_FORCE_FUSED);
-        if (h->pk.r > 0)
+        if (h->pk.r > 0) {
             cands.push_back(path | SPEAR_FORCE_SPLIT);
+            cands.push_back(path | SPEAR_FORCE_FUSED | SPEAR_EC_OFF);
+        }
     }
     cudaEvent_t e0, e1;
     if (cudaEventCreate(&e0) != cudaSuccess)
@@ -533,6 +550,7 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
         cudaEventDestroy(e0);
         return SPEAR_ERR_CUDA;
     }
+    const int b = bucket_of(M);
     float best_ms = 1e30f;
     uint32_t best = 0;
     int rc = SPEAR_OK;
@@ -555,6 +573,11 @@ int spear_w4ec_tune(spear_w4ec *h, const void *x, void *y, int64_t M, void *stre
             break;
         std::sort(times.begin(), times.end());
         const float med = times[times.size() / 2];
+        h->cost_us[b][cost_index(cand)] = med * 1000.0f;
+        if (cand & SPEAR_EC_OFF) {
+            h->cost_us[b][cost_index(cand | SPEAR_FORCE_SPLIT)] = med * 1000.0f;
+            continue;   // a time without the EC, for the cost model only
+        }
         if (med < best_ms) {
             best_ms = med;
             best = cand;

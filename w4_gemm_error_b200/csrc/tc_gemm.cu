@@ -435,8 +435,12 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
             const int lo = ks * p.sps, nm = min(lo + p.sps, p.n_main) - lo;
             const int nst = nm + (ks == p.ksplit - 1 ? p.n_ec : 0);
             const int n = (tile / p.n_ttiles) * BM + i;
+            // the epilogue scales a row whose s is 0 by 1 (its B^T/e operand needs a
+            // nonzero e): such a row dequantises to 0, whatever its codes
+            const bool live = p.s[n] != 0.0f;
             const uint32_t zb = __bfloat16_as_ushort(__float2bfloat16_rn(-(float)(128u + p.z[n])));
-            const uint32_t negz = zb | (zb << 16);
+            const uint32_t negz = live ? (zb | (zb << 16)) : 0u;
+            const uint32_t mulz = live ? 0x3F803F80u : 0u;
             bool ok = true;
             for (int ii = 0; ii < nst; ++ii, ++g) {
                 if ((g & 1u) != grp)
@@ -460,10 +464,10 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                         const int j = 4 * half + jj;
                         // codes k = 8j + {0..7}: nibbles (m, m + 4) hold k = 2m, 2m + 1
                         uint4 o;
-                        o.x = dequant_pair(words[jj], negz);         // k 0, 1
-                        o.y = dequant_pair(words[jj] >> 4, negz);    // k 2, 3
-                        o.z = dequant_pair(words[jj] >> 8, negz);    // k 4, 5
-                        o.w = dequant_pair(words[jj] >> 12, negz);   // k 6, 7
+                        o.x = dequant_pair_mul(words[jj], mulz, negz);         // k 0, 1
+                        o.y = dequant_pair_mul(words[jj] >> 4, mulz, negz);    // k 2, 3
+                        o.z = dequant_pair_mul(words[jj] >> 8, mulz, negz);    // k 4, 5
+                        o.w = dequant_pair_mul(words[jj] >> 12, mulz, negz);   // k 6, 7
                         *reinterpret_cast<uint4 *>(arow + ((j ^ (i & 7)) << 4)) = o;
                     }
                     fence_proxy_async_smem();

@@ -35,7 +35,8 @@ EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_pack_asym", "spe
             "spear_w4ec_destroy", "spear_w4ec_get_packed", "spear_w4ec_get_gate", "spear_w4ec_sync_status",
             "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_gate_noalloc", "spear_w4ec_set_next",
             "spear_w4ec_stack_create", "spear_w4ec_stack_forward", "spear_w4ec_stack_forward_host",
-            "spear_w4ec_stack_buffer", "spear_w4ec_stack_destroy", "spear_w4ec_strerror")
+            "spear_w4ec_stack_buffer", "spear_w4ec_stack_destroy", "spear_w4ec_cost", "spear_w4ec_table_save",
+            "spear_w4ec_table_load", "spear_w4ec_strerror")
 
 
 class SpearError(RuntimeError):
@@ -80,6 +81,9 @@ def _load():
         "spear_w4ec_stack_forward_host": [P, P, P, i64, u32, P],
         "spear_w4ec_stack_buffer": [P, i32, ctypes.POINTER(P)],
         "spear_w4ec_stack_destroy": [P],
+        "spear_w4ec_cost": [P, i64, u32, ctypes.POINTER(f32)],
+        "spear_w4ec_table_save": [P, ctypes.c_char_p, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)],
+        "spear_w4ec_table_load": [P, ctypes.c_char_p],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -194,6 +198,24 @@ def spear_w4ec_gate_noalloc(x, M: int, K: int, w_g, b_g: float, g, stream=None):
            "spear_w4ec_gate_noalloc")
 
 
+def spear_w4ec_cost(h: int, M: int, flags: int) -> float:
+    us = ctypes.c_float(0.0)
+    _check(_lib.spear_w4ec_cost(h, M, flags, ctypes.byref(us)), "spear_w4ec_cost")
+    return us.value
+
+
+def spear_w4ec_table_save(h: int) -> str:
+    n = ctypes.c_size_t(0)
+    _lib.spear_w4ec_table_save(h, None, 0, ctypes.byref(n))
+    buf = ctypes.create_string_buffer(n.value + 1)
+    _check(_lib.spear_w4ec_table_save(h, buf, n.value + 1, ctypes.byref(n)), "spear_w4ec_table_save")
+    return buf.value.decode()
+
+
+def spear_w4ec_table_load(h: int, text: str):
+    _check(_lib.spear_w4ec_table_load(h, text.encode()), "spear_w4ec_table_load")
+
+
 def spear_w4ec_stack_create(ops, max_M: int) -> int:
     """ops: sequence of (layer handle, in, out, ec) tuples."""
     arr = (StackOp * len(ops))(*[StackOp(h, i, o, e) for (h, i, o, e) in ops])
@@ -299,6 +321,16 @@ class W4ECLinear:
 
     def dispatch(self, M: int) -> int:
         return spear_w4ec_dispatch(self.h, M)
+
+    def cost(self, M: int, flags: int) -> float:
+        """Measured microseconds of one forward with these path / placement / EC flags (after tune)."""
+        return spear_w4ec_cost(self.h, M, flags)
+
+    def table_json(self) -> str:
+        return spear_w4ec_table_save(self.h)
+
+    def load_table(self, text: str):
+        spear_w4ec_table_load(self.h, text)
 
     def set_next(self, other: "W4ECLinear | None"):
         """Name the layer whose forward follows this one (prefetch hint; None clears)."""
