@@ -59,7 +59,7 @@ constexpr int kTG = 4;                     // tiles per group
 constexpr int kSubBlocks = 8;             // 64-k sub-blocks of a stage (512 k)
 constexpr int kCW = 2 * kSubBlocks;        // consumer warps: (tile pair, sub-block)
 constexpr int kThreads = 32 * (kCW + 2);   // + producer warp + EC warp
-constexpr int kStageBytes = kTG * 2 * 2048;   // 4 tiles x 2 chunks x (16 rows x 128 B)
+constexpr int kMaxStageChunks = 4;         // 256-k chunks of a stage (one TMA box per tile)
 constexpr int kMaxStages = 16;
 constexpr int kMaxGroups = 16;
 constexpr int kGSlots = 2;                 // G unit buffers, 8 KB each
@@ -86,6 +86,7 @@ struct StreamParams {
     int n_tiles, CS, n_clusters;
     int nch, cpr;          // 256-k chunks of Kp, chunks per rank
     int S;                 // ring stages
+    int sc;                // chunks per stage (a stage is 4 tiles x sc chunks, one box per tile)
     int r, rp, R1p, n_gt;  // n_gt = R1p / 16, 0 without the EC
     int own_max;           // tiles of a group owned by one rank, at most
     int g_slots;           // G unit buffers in use (1 or 2)
@@ -147,7 +148,8 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_
     const int ngroups = (ct + kTG - 1) / kTG;
     const int c_lo = q * p.cpr;
     const int my_ch = max(0, min(p.nch, c_lo + p.cpr) - c_lo);
-    const int nst = (my_ch + 1) / 2;           // stages per group
+    const int nst = (my_ch + p.sc - 1) / p.sc;  // stages per group
+    const uint32_t stage_bytes = (uint32_t)kTG * p.sc * 2048u;
     const int total = ngroups * nst;
     const bool ec = p.n_gt > 0;
     // G units of this rank (16 rows of G x one chunk of its slice), split over the clusters
@@ -200,12 +202,13 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_
                 const int slot = j % p.S, g = j / nst, st = j - g * nst;
                 const int tg = tiles_of(g);
                 const uint32_t bar = smem_addr(&full[slot]);
-                mbar_expect_tx(bar, (uint32_t)tg * 4096u);
-                const uint32_t dst = base + (uint32_t)slot * kStageBytes;
+                mbar_expect_tx(bar, (uint32_t)tg * (uint32_t)p.sc * 2048u);
+                const uint32_t dst = base + (uint32_t)slot * stage_bytes;
                 for (int i = 0; i < tg; ++i) {
+                    // tile t: 16 rows x sc chunks of its row block, one box
                     const int t = t_lo + g * kTG + i;
-                    tma_load_3d(dst + (uint32_t)i * 4096u, &tm_codes, 0, (t & 3) * kTile,
-                                (t >> 2) * p.nch + c_lo + 2 * st, bar);
+                    tma_load_3d(dst + (uint32_t)(i * p.sc) * 2048u, &tm_codes, 0, (t & 3) * kTile,
+                                (t >> 2) * p.nch + c_lo + st * p.sc, bar);
                 }
             };
             const int pre = min(total, p.S);
@@ -447,39 +450,47 @@ decode_stream_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_
                 if (ok)
                     ok = mbar_wait(smem_addr(&full[slot]), (uint32_t)(j / p.S) & 1u, &abort_flag, p.status);
                 if (ok) {
-                    const bool live = sb < 4 * (my_ch - 2 * st);   // a stage may hold one chunk only
-                    uint4 xv[T][2];
-                    const uint8_t *xb = sm + p.off_x + (st * 8 + (live ? sb : 0)) * TOK * 128;
+                    const int nsb = 4 * min(p.sc, my_ch - st * p.sc);   // sub-blocks of this stage
 #pragma unroll
-                    for (int n = 0; n < T; ++n) {
-                        load_x(xb, n, gid, cl, xv[n][0], xv[n][1]);
-                        if (!live)
-                            xv[n][0] = xv[n][1] = make_uint4(0, 0, 0, 0);
-                    }
-                    // codes k = 64 sb + 16 cl + {0..15} of rows gid and gid + 8 of both
-                    // tiles, in chunk sb / 4 of the tile: [16 rows][128 B], 128B swizzle
-                    const int unit = ((2 * (sb & 3) + (cl >> 1)) ^ gid) * 16 + (cl & 1) * 8;
-                    uint2 wgv[2], whv[2];
+                    for (int hh = 0; hh < kMaxStageChunks / 2; ++hh) {
+                        const int sbl = sb + kSubBlocks * hh;
+                        if (hh * kSubBlocks >= 4 * p.sc)
+                            break;
+                        const bool live = sbl < nsb;
+                        uint4 xv[T][2];
+                        const uint8_t *xb = sm + p.off_x + (st * 4 * p.sc + (live ? sbl : 0)) * TOK * 128;
 #pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const uint8_t *ct_ = sm + slot * kStageBytes + ((tp + 2 * i) * 2 + (sb >> 2)) * 2048;
-                        wgv[i] = *reinterpret_cast<const uint2 *>(ct_ + gid * 128 + unit);
-                        whv[i] = *reinterpret_cast<const uint2 *>(ct_ + (gid + 8) * 128 + unit);
-                    }
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
+                        for (int n = 0; n < T; ++n) {
+                            load_x(xb, n, gid, cl, xv[n][0], xv[n][1]);
+                            if (!live)
+                                xv[n][0] = xv[n][1] = make_uint4(0, 0, 0, 0);
+                        }
+                        // codes k = 64 sbl + 16 cl + {0..15} of rows gid and gid + 8 of both
+                        // tiles, in chunk sbl / 4 of the tile's box: [16 rows][128 B], 128B swizzle
+                        const int sbc = live ? sbl : 0;   // a dead sub-block reads valid codes, times zero
+                        const int unit = ((2 * (sbc & 3) + (cl >> 1)) ^ gid) * 16 + (cl & 1) * 8;
+                        uint2 wgv[2], whv[2];
 #pragma unroll
                         for (int i = 0; i < 2; ++i) {
-                            const uint32_t wgw = jj ? wgv[i].y : wgv[i].x, whw = jj ? whv[i].y : whv[i].x;
-                            const uint32_t g0 = dequant_pair(wgw, negg[i]), g1 = dequant_pair(wgw >> 4, negg[i]);
-                            const uint32_t g2 = dequant_pair(wgw >> 8, negg[i]), g3 = dequant_pair(wgw >> 12, negg[i]);
-                            const uint32_t h0 = dequant_pair(whw, negh[i]), h1 = dequant_pair(whw >> 4, negh[i]);
-                            const uint32_t h2 = dequant_pair(whw >> 8, negh[i]), h3 = dequant_pair(whw >> 12, negh[i]);
+                            const uint8_t *ct_ = sm + slot * stage_bytes + ((tp + 2 * i) * p.sc + (sbc >> 2)) * 2048;
+                            wgv[i] = *reinterpret_cast<const uint2 *>(ct_ + gid * 128 + unit);
+                            whv[i] = *reinterpret_cast<const uint2 *>(ct_ + (gid + 8) * 128 + unit);
+                        }
 #pragma unroll
-                            for (int n = 0; n < T; ++n) {
-                                const uint4 v = xv[n][jj];
-                                mma_bf16_16816(acc[jj][i][n], g0, h0, g1, h1, v.x, v.y);
-                                mma_bf16_16816(acc[jj][i][n], g2, h2, g3, h3, v.z, v.w);
+                        for (int jj = 0; jj < 2; ++jj) {
+#pragma unroll
+                            for (int i = 0; i < 2; ++i) {
+                                const uint32_t wgw = jj ? wgv[i].y : wgv[i].x, whw = jj ? whv[i].y : whv[i].x;
+                                const uint32_t g0 = dequant_pair(wgw, negg[i]), g1 = dequant_pair(wgw >> 4, negg[i]);
+                                const uint32_t g2 = dequant_pair(wgw >> 8, negg[i]), g3 = dequant_pair(wgw >> 12, negg[i]);
+                                const uint32_t h0 = dequant_pair(whw, negh[i]), h1 = dequant_pair(whw >> 4, negh[i]);
+                                const uint32_t h2 = dequant_pair(whw >> 8, negh[i]), h3 = dequant_pair(whw >> 12, negh[i]);
+#pragma unroll
+                                for (int n = 0; n < T; ++n) {
+                                    const uint4 v = xv[n][jj];
+                                    mma_bf16_16816(acc[jj][i][n], g0, h0, g1, h1, v.x, v.y);
+                                    mma_bf16_16816(acc[jj][i][n], g2, h2, g3, h3, v.z, v.w);
+                                }
                             }
                         }
                     }
@@ -601,7 +612,7 @@ const void *stream_ptr()
 }
 
 struct StreamPlan {
-    int CS = 0, n_clusters = 0, cpr = 0, S = 0, own_max = 0, btw = 0, ustr = 0, g_slots = 1;
+    int CS = 0, n_clusters = 0, cpr = 0, S = 0, sc = 1, own_max = 0, btw = 0, ustr = 0, g_slots = 1;
     uint32_t off_x = 0, off_red = 0, off_recv = 0, off_g = 0, off_bt = 0, off_u = 0, off_zs = 0;
     size_t smem = 0;
 };
@@ -622,13 +633,14 @@ bool stream_layout(const Packed &pk, int T, int CS, int n_clusters, int S, bool 
     pl.n_clusters = n_clusters;
     pl.cpr = cpr;
     pl.S = S;
+    pl.sc = std::min(cpr, kMaxStageChunks);
     pl.own_max = (kTG + CS - 1) / CS;
     // G units of one CTA at most: 16-row groups of G x chunks of a slice, over the clusters
     const int gu_max = ec ? ((pk.R1p / kTile) * cpr + n_clusters - 1) / n_clusters : 0;
     pl.g_slots = std::max(1, std::min(kGSlots, gu_max));
     pl.btw = pk.rp + 8;
     pl.ustr = pk.rp + 4;
-    size_t off = (size_t)S * kStageBytes;
+    size_t off = (size_t)S * kTG * pl.sc * 2048;
     pl.off_x = (uint32_t)off;
     off += (size_t)4 * cpr * TOK * 128;
     pl.off_red = (uint32_t)off;
@@ -672,7 +684,8 @@ bool stream_plan(const Packed &pk, int64_t M, bool ec, int num_sms, StreamPlan &
         if (best_cost >= 0 && cost >= best_cost)
             continue;
         const int ng_max = (ct_max + kTG - 1) / kTG;
-        const int total = ng_max * ((cpr + 1) / 2);
+        const int sc = std::min(cpr, kMaxStageChunks);
+        const int total = ng_max * ((cpr + sc - 1) / sc);
         StreamPlan pl;
         int S = std::min(total, kMaxStages);
         bool fit = false;
@@ -797,6 +810,17 @@ cudaError_t launch_decode_stream(const Packed &pk, const void *maps, const void 
     StreamPlan pl;
     if (!stream_plan(pk, M, use_ec, num_sms, pl))
         return cudaErrorInvalidValue;
+    // codes as [blocks][64 rows][32 words]: a box is one tile's 16 rows x sc chunks
+    CUtensorMap tm_codes;
+    {
+        const uint64_t dims[3] = {32, 64, (uint64_t)(pk.Np / 64) * (uint64_t)(pk.Kp / 256)};
+        const uint64_t strides[2] = {128, 8192};
+        const uint32_t box[3] = {32, (uint32_t)kTile, (uint32_t)pl.sc};
+        cudaError_t ec_ = make_map_nd(&tm_codes, pk.codes, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, dims, strides, box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+        if (ec_ != cudaSuccess)
+            return ec_;
+    }
     const int T = M <= 8 ? 1 : 2;
     // every cluster must be resident at once
     const int active = max_active_clusters(T, pl.CS, pl.smem);
@@ -843,6 +867,7 @@ cudaError_t launch_decode_stream(const Packed &pk, const void *maps, const void 
     p.nch = (int)(pk.Kp / 256);
     p.cpr = pl.cpr;
     p.S = pl.S;
+    p.sc = pl.sc;
     p.r = pk.r;
     p.rp = pk.rp;
     p.R1p = pk.R1p;
@@ -880,8 +905,8 @@ cudaError_t launch_decode_stream(const Packed &pk, const void *maps, const void 
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     if (T == 1)
-        return cudaLaunchKernelEx(&cfg, decode_stream_kernel<1>, m->codes, m->g, tm_x, p);
-    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<2>, m->codes, m->g, tm_x, p);
+        return cudaLaunchKernelEx(&cfg, decode_stream_kernel<1>, tm_codes, m->g, tm_x, p);
+    return cudaLaunchKernelEx(&cfg, decode_stream_kernel<2>, tm_codes, m->g, tm_x, p);
 }
 
 }  // namespace spear
