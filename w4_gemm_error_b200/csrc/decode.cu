@@ -46,7 +46,9 @@
 //    handle's status word instead of hanging.
 #include <algorithm>
 #include <cstdlib>
+#include <mutex>
 #include <new>
+#include <vector>
 
 #include "async_utils.cuh"
 #include "kernels.h"
@@ -658,11 +660,11 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
 // most 8) whose grid is one wave of two CTAs per SM (so that the next
 // layer's kernel, launched early, also finds room), else CS = 1.  No rank is
 // left without a chunk.  The slice is streamed, so its length is not bounded.
-int pick_cluster(const Packed &pk, int num_sms, int JB, int *KS_out)
+int pick_cluster(const Packed &pk, int num_sms, int JB, int *KS_out, int max_cs = 8)
 {
     const int NC = (int)(pk.Np / kRows);
     const int chunks = (int)(pk.Kp / kChunk);
-    for (int CS = std::min(8, chunks); CS >= 1; --CS) {
+    for (int CS = std::min(max_cs, chunks); CS >= 1; --CS) {
         const int per = (chunks + CS - 1) / CS;
         if (CS > 1 && (CS - 1) * per >= chunks)
             continue;
@@ -726,12 +728,58 @@ bool decode_stream_enabled()
     return v && v[0] == '1';
 }
 
+bool grid_is_one_wave(const void *fn, int threads, size_t smem, int cs, int64_t blocks, int num_sms)
+{
+    struct Entry {
+        const void *fn;
+        int threads, cs, dev;
+        size_t smem;
+        int64_t capacity;
+    };
+    static std::vector<Entry> cache;
+    static std::mutex mu;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const Entry &e : cache)
+            if (e.fn == fn && e.threads == threads && e.cs == cs && e.smem == smem && e.dev == dev)
+                return blocks <= e.capacity;
+    }
+    int64_t capacity = 0;
+    if (raise_smem_limit(fn, smem) == cudaSuccess) {
+        int n = 0;
+        if (cs > 1) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)cs);
+            cfg.blockDim = dim3((unsigned)threads);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = cs;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) == cudaSuccess)
+                capacity = (int64_t)n * cs;
+        } else if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, threads, smem) == cudaSuccess) {
+            capacity = (int64_t)n * num_sms;
+        }
+    }
+    cudaGetLastError();   // a refused query leaves no sticky error
+    std::lock_guard<std::mutex> lock(mu);
+    cache.push_back({fn, threads, cs, dev, smem, capacity});
+    return blocks <= capacity;
+}
+
 bool decode_supported(const Packed &pk, int num_sms)
 {
     if (pk.rp > 128)
         return false;
+    const int JB = pk.r > 0 ? pk.R1p / 16 : 0;
     int KS = 0;
-    const int CS = pick_cluster(pk, num_sms, pk.r > 0 ? pk.R1p / 16 : 0, &KS);
+    const int CS = pick_cluster(pk, num_sms, JB, &KS);
     if (CS == 0)
         return false;
     return plan_for<32>(KS / kChunk, pk.rp, CS, 8).smem <= 227 * 1024;
@@ -824,13 +872,7 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     p.N = pk.N;
     p.JB = use_ec ? pk.R1p / 16 : 0;
     p.NC = (int)(pk.Np / kRows);
-    int KS = 0;
-    const int CS = pick_cluster(pk, num_sms, p.JB, &KS);
-    if (CS == 0)
-        return cudaErrorInvalidValue;
     p.Kp = pk.Kp;
-    p.KS = KS;
-    p.nch = KS / kChunk;
     p.r = pk.r;
     p.rp = use_ec ? pk.rp : 0;
     p.R1p = use_ec ? pk.R1p : 0;
@@ -857,18 +899,36 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     if (e != cudaSuccess)
         return e;
     p.g3 = m->g3;
-    const int W = pick_warps(T, p.nch);
-    const Plan pl = T == 1 ? plan_for<8>(p.nch, p.rp, CS, W)
-                           : (T == 2 ? plan_for<16>(p.nch, p.rp, CS, W) : plan_for<32>(p.nch, p.rp, CS, W));
-    if (pl.smem > 227 * 1024)
-        return cudaErrorInvalidValue;
+    // the largest cluster whose grid is one wave when the EC is on (the row
+    // clusters then wait, bounded, for the EC clusters' partials of u)
+    int CS = 0, W = 0;
+    Plan pl{};
+    const void *fn = nullptr;
+    for (int max_cs = 8; max_cs >= 1;) {
+        int KS = 0;
+        CS = pick_cluster(pk, num_sms, p.JB, &KS, max_cs);
+        if (CS == 0)
+            return cudaErrorInvalidValue;
+        p.KS = KS;
+        p.nch = KS / kChunk;
+        W = pick_warps(T, p.nch);
+        pl = T == 1 ? plan_for<8>(p.nch, p.rp, CS, W)
+                    : (T == 2 ? plan_for<16>(p.nch, p.rp, CS, W) : plan_for<32>(p.nch, p.rp, CS, W));
+        if (pl.smem > 227 * 1024)
+            return cudaErrorInvalidValue;
+        fn = T == 1 ? (W == 16 ? kernel_ptr<1, 16>() : kernel_ptr<1, 8>())
+                    : (T == 2 ? kernel_ptr<2, 8>() : kernel_ptr<4, 8>());
+        e = raise_smem_limit(fn, pl.smem);
+        if (e != cudaSuccess)
+            return e;
+        if (!use_ec || grid_is_one_wave(fn, block_threads(W), pl.smem, CS, (int64_t)(p.JB + p.NC) * CS, num_sms))
+            break;
+        if (CS == 1)
+            return cudaErrorInvalidConfiguration;
+        max_cs = CS - 1;
+    }
     p.S = pl.S;
     p.push = pl.push;
-    const void *fn = T == 1 ? (W == 16 ? kernel_ptr<1, 16>() : kernel_ptr<1, 8>())
-                            : (T == 2 ? kernel_ptr<2, 8>() : kernel_ptr<4, 8>());
-    e = raise_smem_limit(fn, pl.smem);
-    if (e != cudaSuccess)
-        return e;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((p.JB + p.NC) * CS));

@@ -497,7 +497,14 @@ bool decode_rows_shape(const Packed &pk)
 bool decode_rows_fits(const Packed &pk, int64_t M, int num_sms)
 {
     const int64_t ctas = pk.Np / kRowsPerCta + (pk.r > 0 ? (int64_t)pk.R1p / kRowsPerCta * kECSplit : 0);
-    return M >= 1 && M <= kRowsMaxTokens && decode_rows_shape(pk) && ctas <= 2LL * num_sms;
+    if (!(M >= 1 && M <= kRowsMaxTokens && decode_rows_shape(pk) && ctas <= 2LL * num_sms))
+        return false;
+    // the occupancy calculator must agree that the grid is one wave (the row
+    // CTAs wait, bounded, for the CTAs of u)
+    RowsPlan pl;
+    rows_plan(pk, M, pl);
+    const void *fn = pl.T == 1 ? rows_ptr<1, 16, 2>() : rows_ptr<2, 8, 2>();
+    return grid_is_one_wave(fn, 32 * pl.W + 32, pl.smem, 1, ctas, num_sms);
 }
 
 cudaError_t decode_rows_prepare(const Packed &pk, void **maps)

@@ -9,6 +9,14 @@ namespace spear {
 // not a stream operation, and is skipped while a stream is being captured).
 cudaError_t raise_smem_limit(const void *func, size_t bytes);
 
+// Whether `blocks` CTAs of `func` (in clusters of `cs`, 1 for none) with
+// `threads` threads and `smem` bytes of dynamic shared memory can all be
+// resident at once on the current device (the occupancy calculator's answer,
+// cached per kernel, cluster size, shared memory and device).  The decode
+// kernels' CTAs wait on one another with bounded waits, so a grid that is not
+// one wave would only run into those limits.
+bool grid_is_one_wave(const void *func, int threads, size_t smem, int cs, int64_t blocks, int num_sms);
+
 // Library-owned packed layout (all device memory, zero/neutral padded):
 //   codes tiled [Np/64][Kp/256][64][32] uint32: the word holding codes k = 8j..8j+7
 //                             of row n (code of k = 8j+i at bit nibble_shift(i), i.e.

@@ -12,8 +12,11 @@
 // G = [w_g; A^T] (R1p rows), run on the tensor cores with mma.sync: G rows on
 // the 16-row side, 16 tokens per CTA on the 8-column side, the K range split
 // over the CTA's four warps and, when few tokens leave SMs idle, over CTAs.
-// Split-K partials are summed in a fixed order by the last CTA of each token
-// tile to arrive (no floating-point atomics, run-to-run identical).
+// Split-K partials are summed in a fixed order in two levels (no floating-
+// point atomics, run-to-run identical): the last CTA of each group of eight
+// splits to arrive sums the group's partials in split order, and the last
+// group to arrive sums the groups' sums in group order, so no CTA waits on
+// more than eight loads per element.
 #include <algorithm>
 
 #include "async_utils.cuh"
@@ -24,6 +27,9 @@ namespace spear {
 namespace {
 
 constexpr int kTok = 16;  // tokens per CTA (two 8-column MMA tiles)
+constexpr int kGroup = 8;     // splits per first-level sum
+constexpr int kMaxSplits = 32;
+constexpr int kMaxGroups = kMaxSplits / kGroup;
 
 struct PrepassParams {
     const uint16_t *G;
@@ -36,8 +42,10 @@ struct PrepassParams {
     float *v;
     int tf32;
     float *g;
-    float *part;
-    unsigned *counters;
+    float *part;          // [tiles][S][tile] split partials, then [tiles][kMaxGroups][tile] group sums
+    float *gpart;
+    unsigned *counters;   // [tiles] groups summed, then [tiles][kMaxGroups] splits of each group
+    unsigned *gcounters;
     unsigned *ready;   // counted (release) once per token tile when its v is written; null for none
 };
 
@@ -128,37 +136,59 @@ __global__ void __launch_bounds__(128, MINB) prepass_kernel(PrepassParams p)
             mine[e] = red[e];
         __threadfence();
         __syncthreads();
+        const int grp = ks / kGroup, g0 = grp * kGroup, gsize = min(kGroup, p.S - g0);
+        const int ngroups = (p.S + kGroup - 1) / kGroup;
         if (tid == 0)
-            s_last = (atomicAdd(&p.counters[tile], 1u) == (unsigned)(p.S - 1));
+            s_last = (atomicAdd(&p.gcounters[tile * kMaxGroups + grp], 1u) == (unsigned)(gsize - 1));
         __syncthreads();
         if (!s_last)
             return;
         __threadfence();
-        const float *all = p.part + (size_t)tile * p.S * tile_elems;
-        // thread tid sums the elements tid + 128 i (i < 2 MT: the tile is 16 MT x 16)
-        // in split order, loading four partials of all of them per round
+        // first level: this group's partials in split order, four in flight per
+        // round; thread tid takes the elements tid + 128 i (the tile is 16 MT x 16)
+        auto sum_in_order = [&](const float *src, int n, float (&sum)[2 * MT]) {
+#pragma unroll
+            for (int i = 0; i < 2 * MT; ++i)
+                sum[i] = 0.f;
+            for (int q0 = 0; q0 < n; q0 += 4) {
+                float w[4][2 * MT];
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int i = 0; i < 2 * MT; ++i)
+                        w[q][i] = q0 + q < n ? __ldcg(src + (size_t)(q0 + q) * tile_elems + tid + 128 * i) : 0.f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int i = 0; i < 2 * MT; ++i)
+                        sum[i] += w[q][i];
+            }
+        };
         float sum[2 * MT];
+        sum_in_order(p.part + ((size_t)tile * p.S + g0) * tile_elems, gsize, sum);
+        if (tid == 0)
+            p.gcounters[tile * kMaxGroups + grp] = 0u;
+        if (ngroups > 1) {
+            // second level: the groups' sums in group order, by the last group
+            float *gdst = p.gpart + ((size_t)tile * kMaxGroups + grp) * tile_elems;
 #pragma unroll
-        for (int i = 0; i < 2 * MT; ++i)
-            sum[i] = 0.f;
-        for (int q0 = 0; q0 < p.S; q0 += 4) {
-            float w[4][2 * MT];
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int i = 0; i < 2 * MT; ++i)
-                    w[q][i] = q0 + q < p.S ? __ldcg(all + (size_t)(q0 + q) * tile_elems + tid + 128 * i) : 0.f;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-#pragma unroll
-                for (int i = 0; i < 2 * MT; ++i)
-                    sum[i] += w[q][i];
+            for (int i = 0; i < 2 * MT; ++i)
+                gdst[tid + 128 * i] = sum[i];
+            __threadfence();
+            __syncthreads();
+            if (tid == 0)
+                s_last = (atomicAdd(&p.counters[tile], 1u) == (unsigned)(ngroups - 1));
+            __syncthreads();
+            if (!s_last)
+                return;
+            __threadfence();
+            sum_in_order(p.gpart + (size_t)tile * kMaxGroups * tile_elems, ngroups, sum);
+            if (tid == 0)
+                p.counters[tile] = 0u;
         }
 #pragma unroll
         for (int i = 0; i < 2 * MT; ++i)
             red[tid + 128 * i] = sum[i];
-        if (tid == 0)
-            p.counters[tile] = 0u;
         __syncthreads();
     }
 
@@ -192,7 +222,7 @@ int pick_splits(int64_t M, int64_t Kp, int num_sms)
     const int nkb = (int)(Kp / 64);
     int S = std::max(1, (2 * num_sms) / std::max(tiles, 1));
     S = std::min(S, std::max(1, nkb / 4));  // at least one k block per warp
-    return std::min(S, 32);                  // the last CTA sums them four at a time
+    return std::min(S, kMaxSplits);          // summed in groups of eight
 }
 
 using PrepassFn = void (*)(PrepassParams);
@@ -220,18 +250,20 @@ size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms)
 {
     size_t worst = 0;
     // the split count shrinks as M grows; check every tile count up to max_M
+    // (split partials, then kMaxGroups group sums per tile)
     const int64_t tiles_max = (max_M + kTok - 1) / kTok;
     for (int64_t tiles = 1; tiles <= tiles_max; ++tiles) {
         const int S = pick_splits(tiles * kTok, pk.Kp, num_sms);
         if (S > 1)
-            worst = std::max(worst, (size_t)tiles * S * pk.R1p * kTok);
+            worst = std::max(worst, (size_t)tiles * (S + kMaxGroups) * pk.R1p * kTok);
         else
             break;
     }
     return worst;
 }
 
-int prepass_counters(int64_t max_M) { return (int)((max_M + kTok - 1) / kTok); }
+// One counter per token tile for the groups, then kMaxGroups per tile for the splits.
+int prepass_counters(int64_t max_M) { return (int)((max_M + kTok - 1) / kTok) * (1 + kMaxGroups); }
 
 cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
                            const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready, bool slim)
@@ -255,11 +287,14 @@ cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v,
     p.v = v;
     p.tf32 = tf32 ? 1 : 0;
     p.g = g;
-    p.part = w.part;
-    p.counters = w.counters;
-    p.ready = ready;
     const int tiles = (int)((M + kTok - 1) / kTok);
-    if (tiles > w.n_counters || (p.S > 1 && (size_t)tiles * p.S * pk.R1p * kTok > w.part_floats))
+    const int tiles_cap = w.n_counters / (1 + kMaxGroups);
+    p.part = w.part;
+    p.gpart = w.part + (size_t)tiles * p.S * pk.R1p * kTok;
+    p.counters = w.counters;
+    p.gcounters = w.counters + tiles_cap;
+    p.ready = ready;
+    if (tiles > tiles_cap || (p.S > 1 && (size_t)tiles * (p.S + kMaxGroups) * pk.R1p * kTok > w.part_floats))
         return cudaErrorInvalidValue;
     PrepassFn fn = prepass_fn(pk.R1p / 16, slim);
     if (!fn)
