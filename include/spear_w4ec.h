@@ -70,7 +70,9 @@ enum {
                                  one CTA per 16 weight rows over all of K (up to 16 tokens, K a
                                  multiple of 64 and at most 8192, one wave of CTAs), else the
                                  split-K streaming kernel (up to 32 tokens per launch) */
-    SPEAR_FORCE_TC = 16u      /* tcgen05 / TMEM tile kernel (larger M) */
+    SPEAR_FORCE_TC = 16u,     /* tcgen05 / TMEM tile kernel (larger M) */
+    SPEAR_STACK_PERSISTENT = 32u /* spear_w4ec_stack_forward only: run the whole stack as one
+                                 persistent kernel (up to 16 tokens; see the stack section) */
 };
 
 typedef struct spear_w4ec_opts {
@@ -286,7 +288,20 @@ int spear_w4ec_stack_create(spear_w4ec_stack **out, const spear_w4ec_stack_op *o
  * spear_w4ec_forward on the same input with flags 0 (EC placed) or
  * SPEAR_EC_OFF (EC not placed), bit for bit.  `flags` (0 for the placement
  * as given) may add SPEAR_FORCE_* path flags or SPEAR_EC_OFF, which then
- * apply to every op. */
+ * apply to every op.
+ *
+ * With SPEAR_STACK_PERSISTENT (and optionally SPEAR_EC_OFF, no path flag)
+ * the ops run instead as ONE kernel launch of one CTA per SM that stays
+ * resident for the whole stack (plus a clear of its counters before it): the
+ * weights of later ops stream into shared memory while earlier ops compute,
+ * and an op waits (bounded, on device counters) only for the earlier op it
+ * depends on.  For M <= 16 on stacks whose layers all have K a multiple of 8
+ * and r <= 64; otherwise SPEAR_ERR_UNSUPPORTED.  Its results match the same
+ * definition within the same fp32-accumulation bounds, not bit for bit: the
+ * EC down-projection of an op that reads the previous op's output is summed
+ * from that op's epilogues with fp32 atomic adds (order may vary run to run).
+ * A wait that runs out sets the timeout bit of the status word of the layer
+ * of the op that waited (spear_w4ec_sync_status). */
 int spear_w4ec_stack_forward(spear_w4ec_stack *s, const void *x, void *y, int64_t M, uint32_t flags,
                              void *stream);
 

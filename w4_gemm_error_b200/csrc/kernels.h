@@ -1,5 +1,6 @@
 // Launch interfaces of the kernels behind the C ABI (library-internal).
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -125,6 +126,41 @@ cudaError_t decode_stream_prepare(const Packed &pk, void **maps);
 void decode_stream_free(void *maps);
 cudaError_t launch_decode_stream(const Packed &pk, const void *maps, const void *x, void *y, int64_t M, bool ec,
                                  const DecodeWork &w, int *status, cudaStream_t st, int num_sms);
+
+// ---- persistent decode kernel over a whole layer stack (up to 16 tokens, one
+// CTA per SM for the whole stack; see stack_decode.cu).  The stack builds one
+// StackOpDev per op (device memory) and two tensor maps per op.
+constexpr int kStackMaxTokens = 16;
+constexpr int kStackMaxRp = 64;
+constexpr int kStackMaxR1p = 80;
+struct StackOpDev {
+    const float *s;
+    const uint8_t *z;
+    const uint16_t *Bt;
+    const uint16_t *Gnext;   // G of the next op (its u is formed in this op's epilogue), or null
+    const uint16_t *xbuf;    // input buffer (null: the call's x)
+    uint16_t *ybuf;          // output buffer (null: the call's y)
+    int *status;             // status word of the op's layer
+    int K, N, nch, rp, R1p;
+    int R1p_next, Kp_next;
+    float b_g;
+    int ec;                  // EC placed (and the layer has one)
+    int u_mode;              // 0 no EC; 1 u from this op's EC units; 2 u from the previous op's epilogues
+    int fuse_next;           // this op's epilogues form the next op's u
+    int wait_op;             // the latest earlier op this one conflicts with (-1: none)
+    int base;                // CTA that takes this op's item 0
+    int n_g, n_tiles;        // EC units (u_mode 1) and 16-row tiles
+    int u_off;               // float offset of the op's u accumulator [R1p][16]
+};
+bool stack_decode_layer_ok(const Packed &pk);
+bool stack_decode_fits(int num_sms);
+cudaError_t stack_decode_maps(const Packed &pk, CUtensorMap *codes, CUtensorMap *g);
+// done: [2 n_ops] counters followed by the u accumulators, ws_bytes in all
+// (cleared on the stream before the kernel); fault: make the first wait run
+// out (fault injection of the timeout path).
+cudaError_t launch_stack_decode(const StackOpDev *ops, const CUtensorMap *maps, int n_ops, const void *x, void *y,
+                                int64_t M, bool ec_on, unsigned *done, float *uacc, size_t ws_bytes, bool fault,
+                                cudaStream_t st, int num_sms);
 
 // ---- split EC: y[t][n] = bf16(y[t][n] + sum_j v[t][j] * Bt[n][j]), v in fp32
 cudaError_t launch_ec_apply(const Packed &pk, const float *vf, void *y, int64_t M, cudaStream_t st);

@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "handle.h"
+#include "tensor_map.h"
 #include "spear_w4ec.h"
 
 using namespace spear;
@@ -26,6 +27,14 @@ struct spear_w4ec_stack {
     int64_t out_width = 0;      // N of the last op
     void *x_stage = nullptr;    // staging of the host-buffer call
     void *y_stage = nullptr;
+    // the persistent decode kernel's plan (stack_decode.cu), when every op fits it
+    bool persist = false;
+    int num_sms = 0;
+    bool fault_launch = false, fault_timeout = false;
+    spear::StackOpDev *p_ops = nullptr;    // device [n_ops]
+    CUtensorMap *p_maps = nullptr;         // device [n_ops][2]
+    unsigned *p_ws = nullptr;              // device: [2 n_ops] counters, then the u accumulators
+    size_t p_ws_bytes = 0;
 };
 
 namespace {
@@ -38,12 +47,117 @@ void free_stack(spear_w4ec_stack *s)
         cudaFree(b);
     cudaFree(s->x_stage);
     cudaFree(s->y_stage);
+    cudaFree(s->p_ops);
+    cudaFree(s->p_maps);
+    cudaFree(s->p_ws);
+}
+
+// The persistent kernel's plan: per op its operands, buffers, the op it must
+// wait for (the latest earlier op that writes what it reads, or reads or
+// writes what it writes), where its u comes from, and where the round-robin
+// deal of its items starts.  Leaves s->persist false (and allocates nothing)
+// when some op does not fit the kernel.
+cudaError_t plan_persistent(spear_w4ec_stack *s)
+{
+    const int n = (int)s->ops.size();
+    s->num_sms = s->ops[0].layer->num_sms;
+    for (const spear_w4ec_stack_op &op : s->ops)
+        if (!stack_decode_layer_ok(op.layer->pk))
+            return cudaSuccess;
+    if (!tensor_maps_available() || !stack_decode_fits(s->num_sms))
+        return cudaSuccess;
+    std::vector<StackOpDev> dev(n);
+    std::vector<CUtensorMap> maps(2 * (size_t)n);
+    auto ec_of = [&](int l) { return s->ops[l].ec && s->ops[l].layer->pk.r > 0; };
+    int64_t base = 0, u_floats = 0;
+    for (int l = 0; l < n; ++l) {
+        const spear_w4ec_stack_op &op = s->ops[l];
+        const Packed &pk = op.layer->pk;
+        StackOpDev &d = dev[l];
+        d = StackOpDev{};
+        d.s = pk.s;
+        d.z = pk.z;
+        d.Bt = pk.Bt;
+        d.xbuf = op.in == 0 ? nullptr : static_cast<const uint16_t *>(s->bufs[op.in]);
+        d.ybuf = op.out == 1 ? nullptr : static_cast<uint16_t *>(s->bufs[op.out]);
+        d.status = op.layer->status;
+        d.K = (int)pk.K;
+        d.N = (int)pk.N;
+        d.nch = (int)(pk.Kp / 256);
+        d.rp = pk.rp;
+        d.R1p = pk.R1p;
+        d.b_g = pk.b_g;
+        d.ec = ec_of(l) ? 1 : 0;
+        d.wait_op = -1;
+        for (int j = l - 1; j >= 0 && d.wait_op < 0; --j) {
+            const spear_w4ec_stack_op &o = s->ops[j];
+            if (o.out == op.in || o.in == op.out || o.out == op.out)
+                d.wait_op = j;
+        }
+        const bool chained = l > 0 && s->ops[l - 1].out == op.in;
+        d.u_mode = !d.ec ? 0 : (chained ? 2 : 1);
+        if (l + 1 < n && ec_of(l + 1) && s->ops[l + 1].in == op.out) {
+            const Packed &nx = s->ops[l + 1].layer->pk;
+            d.fuse_next = 1;
+            d.Gnext = nx.G;
+            d.R1p_next = nx.R1p;
+            d.Kp_next = (int)nx.Kp;
+        }
+        d.n_g = d.u_mode == 1 ? pk.R1p / 16 * d.nch : 0;
+        d.n_tiles = (int)((pk.N + 15) / 16);
+        d.base = (int)(base % s->num_sms);
+        base += d.n_g + d.n_tiles;
+        if (d.ec) {
+            d.u_off = (int)u_floats;
+            u_floats += (int64_t)pk.R1p * 16;
+        }
+        cudaError_t e = stack_decode_maps(pk, &maps[2 * l], &maps[2 * l + 1]);
+        if (e != cudaSuccess)
+            return e;
+    }
+    s->p_ws_bytes = (size_t)2 * n * sizeof(unsigned) + (size_t)u_floats * sizeof(float);
+    s->p_ws_bytes = (s->p_ws_bytes + 15) / 16 * 16;
+    cudaError_t e = cudaMalloc(&s->p_ops, sizeof(StackOpDev) * n);
+    if (e == cudaSuccess)
+        e = cudaMalloc(&s->p_maps, sizeof(CUtensorMap) * 2 * (size_t)n);
+    if (e == cudaSuccess)
+        e = cudaMalloc(&s->p_ws, s->p_ws_bytes);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(s->p_ops, dev.data(), sizeof(StackOpDev) * n, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+        e = cudaMemcpy(s->p_maps, maps.data(), sizeof(CUtensorMap) * 2 * (size_t)n, cudaMemcpyHostToDevice);
+    if (e != cudaSuccess)
+        return e;
+    for (const spear_w4ec_stack_op &op : s->ops) {
+        s->fault_launch = s->fault_launch || op.layer->fault_launch;
+        s->fault_timeout = s->fault_timeout || op.layer->fault_timeout;
+    }
+    s->persist = true;
+    return cudaSuccess;
+}
+
+constexpr uint32_t kPathFlags = SPEAR_FORCE_FUSED | SPEAR_FORCE_SPLIT | SPEAR_FORCE_DECODE | SPEAR_FORCE_TC;
+
+int run_persistent(spear_w4ec_stack *s, const void *x, void *y, int64_t M, uint32_t flags, cudaStream_t st)
+{
+    if (!s->persist || M > kStackMaxTokens || (flags & kPathFlags))
+        return SPEAR_ERR_UNSUPPORTED;
+    if (s->fault_launch)
+        return SPEAR_ERR_CUDA;
+    unsigned *done = s->p_ws;
+    float *uacc = reinterpret_cast<float *>(s->p_ws + 2 * s->ops.size());
+    const cudaError_t e = launch_stack_decode(s->p_ops, s->p_maps, (int)s->ops.size(), x, y, M,
+                                              !(flags & SPEAR_EC_OFF), done, uacc, s->p_ws_bytes, s->fault_timeout,
+                                              st, s->num_sms);
+    return e == cudaSuccess ? SPEAR_OK : status_of(e);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int run_ops(spear_w4ec_stack *s, const void *x, void *y, int64_t M, uint32_t flags, cudaStream_t st)
 {
+    if (flags & SPEAR_STACK_PERSISTENT)
+        return run_persistent(s, x, y, M, flags & ~(uint32_t)SPEAR_STACK_PERSISTENT, st);
     for (const spear_w4ec_stack_op &op : s->ops) {
         const void *in = op.in == 0 ? x : s->bufs[op.in];
         void *out = op.out == 1 ? y : s->bufs[op.out];
@@ -118,6 +232,8 @@ int spear_w4ec_stack_create(spear_w4ec_stack **out, const spear_w4ec_stack_op *o
         e = cudaMalloc(&s->x_stage, (size_t)max_M * (size_t)in_width * 2);
     if (e == cudaSuccess)
         e = cudaMalloc(&s->y_stage, (size_t)max_M * (size_t)s->out_width * 2);
+    if (e == cudaSuccess)
+        e = plan_persistent(s);
     if (e != cudaSuccess) {
         free_stack(s);
         delete s;

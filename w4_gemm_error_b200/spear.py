@@ -29,6 +29,7 @@ SPEAR_FORCE_FUSED = 2
 SPEAR_FORCE_SPLIT = 4
 SPEAR_FORCE_DECODE = 8
 SPEAR_FORCE_TC = 16
+SPEAR_STACK_PERSISTENT = 32   # stack forward only: one persistent kernel for the whole stack
 
 EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_pack_asym", "spear_w4ec_import",
             "spear_w4ec_forward", "spear_w4ec_forward_host",
