@@ -416,8 +416,14 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             mine[(gid + 8) * TOK + col + 1] = acc[n][3];
         }
     }
-    if (!ok)
+    __shared__ int s_gave_up;   // some wait of this CTA ran out
+    if (tid == 0)
+        s_gave_up = 0;
+    __syncthreads();
+    if (!ok) {
         atomicOr(p.status, kStatusTimeout);
+        s_gave_up = 1;
+    }
     __syncthreads();
     if (tid < kConsumers) {
         if (!is_u) {
@@ -438,15 +444,20 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             }
         }
     } else if (lane == 0) {
-        // no copy of this CTA may still be landing when it goes on (bounded;
-        // immediate unless a wait gave up): stages reused before the last S
-        // chunks were released by the consumers after they landed
-        for (int c = max(0, issued - S); c < issued; ++c) {
-            wait_bounded(bar_full_w + 8 * (c % S), (uint32_t)(c / S) & 1u);
-            wait_bounded(bar_full_x + 8 * (c % S), (uint32_t)(c / S) & 1u);
+        // no copy of this CTA may still be landing when it goes on (bounded).
+        // Every stage the producer filled was waited for by the consumers
+        // unless one of their waits gave up; only then are the stages waited
+        // for here (each mbarrier test costs hundreds of cycles: the 2S tests
+        // took about 2.5 us per launch).  B^T is waited for only by an
+        // epilogue with the EC, so always here.
+        if (s_gave_up) {
+            for (int c = max(0, issued - S); c < issued; ++c) {
+                wait_bounded(bar_full_w + 8 * (c % S), (uint32_t)(c / S) & 1u);
+                wait_bounded(bar_full_x + 8 * (c % S), (uint32_t)(c / S) & 1u);
+            }
+            for (int c = issued; c < first; ++c)   // codes requested, activations never
+                wait_bounded(bar_full_w + 8 * c, 0);
         }
-        for (int c = issued; c < first; ++c)   // codes requested, activations never
-            wait_bounded(bar_full_w + 8 * c, 0);
         if (!is_u && rank == 0 && p.rp > 0)
             wait_bounded(bar_bt, 0);
     }

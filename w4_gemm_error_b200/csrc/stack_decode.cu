@@ -238,9 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1) stack_decode_kernel(StackParams p
                     }
             }
         }
-        // no copy may still be landing when the CTA leaves: wait for the last
-        // phase issued on every stage and operand slot
-        if (lane == 0) {
+        // no copy may still be landing when the CTA leaves: the consumers waited
+        // for every stage and operand slot issued unless a wait gave up; then the
+        // last phase issued on each is waited for here
+        if (lane == 0 && *abrt) {
             for (uint32_t q = rseq > (uint32_t)kStages ? rseq - kStages : 0; q < rseq; ++q)
                 mbar_wait_final(smem_addr(&full[q % kStages]), (q / kStages) & 1);
             for (uint32_t q = mseq > (uint32_t)kMetaSlots ? mseq - kMetaSlots : 0; q < mseq; ++q)

@@ -178,10 +178,12 @@ tc_prepass_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constan
                 tma_load_2d(sb, &tm_x, kb * 64, t0, full0 + 8 * slot);
                 tma_load_2d(sb + x_bytes, &tm_g, kb * 64, 0, full0 + 8 * slot);
             }
-            for (int k = 0; k < PP_STAGES && k < issued; ++k) {
-                const int kb = issued - 1 - k;
-                mbar_wait_final(full0 + 8 * (kb % PP_STAGES), (kb / PP_STAGES) & 1);
-            }
+            // (the MMA thread waited for every stage issued unless a wait gave up)
+            if (abort_flag)
+                for (int k = 0; k < PP_STAGES && k < issued; ++k) {
+                    const int kb = issued - 1 - k;
+                    mbar_wait_final(full0 + 8 * (kb % PP_STAGES), (kb / PP_STAGES) & 1);
+                }
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -360,11 +362,13 @@ tc_w4ec_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__
                     }
                 }
             }
-            // do not leave while copies this CTA issued may still land
-            for (uint32_t k = 0; k < STAGES && k < g; ++k) {
-                const uint32_t gg = g - 1 - k, slot = gg % STAGES, phase = (gg / STAGES) & 1;
-                mbar_wait_final(full0 + 8 * slot, phase);
-            }
+            // do not leave while copies this CTA issued may still land (the
+            // consumers waited for every stage unless a wait gave up)
+            if (abort_flag)
+                for (uint32_t k = 0; k < STAGES && k < g; ++k) {
+                    const uint32_t gg = g - 1 - k, slot = gg % STAGES, phase = (gg / STAGES) & 1;
+                    mbar_wait_final(full0 + 8 * slot, phase);
+                }
             // early start: this grid completes only after its predecessor (the
             // prepass), so that the next kernel's wait still covers both
             if (p.v_ready)
