@@ -61,6 +61,7 @@ constexpr int kRows = 64;         // weight rows per cluster (four warps x 16)
 constexpr int kChunk = 256;       // k per stage (one 8 KB TMA box of 64 rows of codes)
 constexpr int kMaxStages = 8;     // ring depth limit
 constexpr int kUStride = 32;      // token stride of the published u rows
+constexpr int kUFinal = 8;        // slot of ws_u holding the summed u (slots 0..7: partials)
 // A CTA has W consumer warps, W = 16 (one per 16-row group and 64-k
 // sub-block of a stage) or W = 8 (two sub-blocks each), then one producer warp.
 __host__ __device__ constexpr int block_threads(int W) { return 32 * W + 32; }
@@ -88,6 +89,8 @@ struct DecodeParams {
     int KS, nch;          // k per CTA (a multiple of 256), chunks of 256 k per CTA
     int S;                // ring stages
     int JB, NC;           // EC clusters, 64-row clusters
+    int ES;               // EC clusters per 16 rows of G (each a 1/ES share of K): JB = R1p/16 * ES
+    int KSe, nche;        // k per EC CTA (a multiple of 256), its chunks of 256 k
     int r, rp, R1p;
     int push;             // partial tiles pushed into receive slots of the first CTA
     int x3, g3;           // activations / G rows as one 3-D box per stage (else four 2-D boxes)
@@ -176,9 +179,12 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     const uint32_t rank = cluster_ctarank();
     const int cluster = blockIdx.x / CS;
     const bool is_u = cluster < p.JB;
-    const int k0 = (int)rank * p.KS;
+    // an EC CTA takes rows 16 jg .. + 15 of G over slice sl of K (ES x CS slices)
+    const int jg = is_u ? cluster / p.ES : 0;
+    const int sl = is_u ? (cluster % p.ES) * CS + (int)rank : (int)rank;
+    const int k0 = sl * (is_u ? p.KSe : p.KS);
     // the last ranks may hold a shorter (or empty) slice when K/256 is not a multiple of CS
-    const int nch = max(0, min(p.nch, (int)((p.Kp - k0) / kChunk)));
+    const int nch = max(0, min(is_u ? p.nche : p.nch, (int)((p.Kp - k0) / kChunk)));
     const int S = p.S;
     const int first = min(S, nch);   // chunks whose stages are filled before the dependency wait
     const uint32_t bar_full_w = smem_addr(&bars[0]);
@@ -202,10 +208,10 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         mbar_expect_tx(bar, 8192);
         if (is_u) {
             if (p.g3)
-                tma_load_3d(dst, &tm_g, 0, 16 * cluster, (k0 + c * kChunk) / 64, bar);
+                tma_load_3d(dst, &tm_g, 0, 16 * jg, (k0 + c * kChunk) / 64, bar);
             else
                 for (int i = 0; i < 4; ++i)
-                    tma_load_2d(dst + i * 2048, &tm_g, k0 + c * kChunk + i * 64, 16 * cluster, bar);
+                    tma_load_2d(dst + i * 2048, &tm_g, k0 + c * kChunk + i * 64, 16 * jg, bar);
         } else {
             tma_load_3d(dst, &tm_codes, 0, 0, (n0 / kRows) * (int)(p.Kp / kChunk) + (k0 / kChunk) + c, bar);
         }
@@ -265,6 +271,48 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
         for (int i = 0; i < 4; ++i)
             acc[n][i] = acc2[n][i] = 0.f;
 
+    constexpr bool kOverlap = W == 16;
+    constexpr int kSumThreads = kOverlap ? 128 : kConsumers - 32;
+    const bool fetcher = kOverlap && rank == 0 && p.JB > 0 && tid >= kSumThreads && tid < kConsumers;
+    const int nsum = (p.JB > 0 && kOverlap) ? kSumThreads : kConsumers;   // summing threads: tid < nsum
+    constexpr int tile4 = kRows * TOK / 4;
+    float *u0 = reinterpret_cast<float *>(bp + L.u);
+    float *uT = u0 + TOK;
+    const int nparts = CS * p.ES;   // partials of u, one per slice of K (at most 8)
+    // u (the final rows, four tokens per load, every load of a round issued
+    // before any is used) into u0 and uT
+    auto fetch_u = [&](int ft, int nft, bool good) {
+        constexpr int kT4 = TOK / 4;
+        const int n4 = (1 + p.r) * kT4;
+        const float *fin = p.ws_u + (int64_t)kUFinal * p.R1p * kUStride;
+        for (int e0 = ft; e0 < n4; e0 += 4 * nft) {
+            float4 v[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = e0 + i * nft, row = e / kT4, t4 = e - row * kT4;
+                v[i] = (e < n4 && good) ? __ldcg(reinterpret_cast<const float4 *>(fin + row * kUStride + 4 * t4))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int e = e0 + i * nft, row = e / kT4, t4 = e - row * kT4;
+                if (e >= n4)
+                    continue;
+                const float uu[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (row == 0)
+                        u0[4 * t4 + c] = uu[c];
+                    else
+                        uT[(4 * t4 + c) * p.rp + row - 1] = uu[c];
+                }
+            }
+        }
+        for (int e = ft; e < TOK * (p.rp - p.r); e += nft) {
+            const int t = e / (p.rp - p.r), j = p.r + e - t * (p.rp - p.r);
+            uT[t * p.rp + j] = 0.f;
+        }
+    };
     float *red = reinterpret_cast<float *>(bp + L.red);
     if (producer) {
         if (lane == 0) {
@@ -289,6 +337,15 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             prefetch_l2_share(p.pf, p.pf_bytes);
         }
         __syncwarp();
+        if (!kOverlap && !is_u && rank == 0 && p.JB > 0) {
+            // with 8 consumer warps: u (summed over its partials) goes into shared
+            // memory while the consumers finish their stages
+            int good = 1;
+            if (lane == 0)
+                good = wait_u_published(p, (unsigned)(p.JB / p.ES)) ? 1 : 0;
+            good = __shfl_sync(0xffffffffu, good, 0);
+            fetch_u(lane, 32, good != 0);
+        }
     } else if (!is_u) {
         // ---- 64 weight rows: warp w owns rows 16(w mod 4) .. +15 and the sub-blocks
         // sb = w/4 (mod KPAR) of each stage
@@ -465,61 +522,55 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     __syncthreads();
 
     if (is_u) {
-        // ---- publish this CTA's partial of u rows 16*cluster .. +15 (all TOK
-        // columns); the 64-row clusters sum the CS partials in rank order
-        float *dst = p.ws_u + ((int64_t)rank * p.R1p + 16 * cluster) * kUStride;
+        // ---- publish this CTA's partial of u rows 16 jg .. + 15 (all TOK
+        // columns); the EC CTA of the group that arrives last sums the ES x CS
+        // partials in slice order into the final rows (slot 8 of ws_u) and
+        // counts the group published, so that a row cluster reads u once
+        float *dst = p.ws_u + ((int64_t)sl * p.R1p + 16 * jg) * kUStride;
         for (int e = tid; e < 16 * TOK; e += kThreads) {
             const int row = e / TOK, t = e - row * TOK;
             dst[row * kUStride + t] = red[e];
         }
+        __shared__ int s_last;
         __syncthreads();
-        if (tid == 0)
-            red_release_gpu_add(&p.flags[0], 1u);
+        if (tid == 0) {
+            __threadfence();
+            s_last = atomicAdd(&p.flags[2 + jg], 1u) == (unsigned)(nparts - 1) ? 1 : 0;
+        }
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            for (int e = tid; e < 16 * TOK; e += kThreads) {
+                const int row = e / TOK, t = e - row * TOK;
+                float v[8];
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    v[q] = q < nparts ? __ldcg(p.ws_u + ((int64_t)q * p.R1p + 16 * jg + row) * kUStride + t) : 0.f;
+                float u = v[0];
+#pragma unroll
+                for (int q = 1; q < 8; ++q)
+                    if (q < nparts)
+                        u += v[q];
+                p.ws_u[((int64_t)kUFinal * p.R1p + 16 * jg + row) * kUStride + t] = u;
+            }
+            __syncthreads();
+            if (tid == 0) {
+                p.flags[2 + jg] = 0u;
+                red_release_gpu_add(&p.flags[0], 1u);
+            }
+        }
         if (push && !solo)
             cluster_wait();   // pairs with the arrive after the barrier set-up
         return;
     }
 
     // ---- sum the K split over the cluster, in rank order, in the first CTA.
-    // With an EC, u is published by the EC clusters as CS partials, which are
-    // summed (rank order) into u0 [TOK] (gate logits) and uT [TOK][rp]
-    // (u[1 + j][t] transposed, zero for j >= r): with 16 consumer warps, warps
-    // 0-3 sum the K split while the other twelve wait for u and fetch it; with
-    // 8, the last consumer warp waits for u during the sum and every consumer
-    // thread fetches it afterwards (a fetch by half of the threads needs more
-    // round trips than the overlap saves).  The producer warp only takes part
-    // in the barriers.
-    constexpr bool kOverlap = W == 16;
-    constexpr int kSumThreads = kOverlap ? 128 : kConsumers - 32;
-    const bool fetcher = kOverlap && rank == 0 && p.JB > 0 && tid >= kSumThreads && tid < kConsumers;
-    const bool poller = !kOverlap && rank == 0 && p.JB > 0 && warp == W - 1;
-    const int nsum = p.JB > 0 ? kSumThreads : kConsumers;   // summing threads: tid < nsum
-    __shared__ int s_good;
-    constexpr int tile4 = kRows * TOK / 4;
-    float *u0 = reinterpret_cast<float *>(bp + L.u);
-    float *uT = u0 + TOK;
-    auto fetch_u = [&](int ft, int nft, bool good) {
-        for (int e = ft; e < (1 + p.r) * TOK; e += nft) {
-            const int row = e / TOK, t = e - row * TOK;
-            float v[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q)
-                v[q] = (q < CS && good) ? __ldcg(p.ws_u + ((int64_t)q * p.R1p + row) * kUStride + t) : 0.f;
-            float u = v[0];
-#pragma unroll
-            for (int q = 1; q < 8; ++q)
-                if (q < CS)
-                    u += v[q];
-            if (row == 0)
-                u0[t] = u;
-            else
-                uT[t * p.rp + row - 1] = u;
-        }
-        for (int e = ft; e < TOK * (p.rp - p.r); e += nft) {
-            const int t = e / (p.rp - p.r), j = p.r + e - t * (p.rp - p.r);
-            uT[t * p.rp + j] = 0.f;
-        }
-    };
+    // With an EC, u is published by the EC CTAs as ES x CS partials (one per
+    // slice of K), which are summed (slice order) into u0 [TOK] (gate logits)
+    // and uT [TOK][rp] (u[1 + j][t] transposed, zero for j >= r): with 16
+    // consumer warps, warps 0-3 sum the K split while the other twelve wait
+    // for u and fetch it; with 8, the producer warp has fetched it while the
+    // consumers ran their last stages (above).
     if (push) {
         if (!solo)
             cluster_wait();   // every receive barrier of the cluster is initialised
@@ -532,19 +583,16 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             cluster_wait();   // the first CTA has received every tile
             return;
         }
-        if (!fetcher && !poller && CS > 1 && !wait_bounded(bar_recv, 0) && tid == 0)
+        if (!fetcher && CS > 1 && !wait_bounded(bar_recv, 0) && tid == 0)
             atomicOr(p.status, kStatusTimeout);
         if (!solo)
             cluster_arrive();     // the tiles have landed: the other CTAs may leave
-        if (fetcher || poller) {
+        if (fetcher) {
             int good = 1;
             if (lane == 0)
-                good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
+                good = wait_u_published(p, (unsigned)(p.JB / p.ES)) ? 1 : 0;
             good = __shfl_sync(0xffffffffu, good, 0);
-            if (fetcher)
-                fetch_u(tid - kSumThreads, kConsumers - kSumThreads, good != 0);
-            else if (lane == 0)
-                s_good = good;
+            fetch_u(tid - kSumThreads, kConsumers - kSumThreads, good != 0);
         }
         const float4 *slots = reinterpret_cast<const float4 *>(bp + L.recv);
         if (tid < nsum)
@@ -562,15 +610,12 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
     } else {
         if (!solo)
             cluster_sync();
-        if (fetcher || poller) {
+        if (fetcher) {
             int good = 1;
             if (lane == 0)
-                good = wait_u_published(p, (unsigned)(p.JB * CS)) ? 1 : 0;
+                good = wait_u_published(p, (unsigned)(p.JB / p.ES)) ? 1 : 0;
             good = __shfl_sync(0xffffffffu, good, 0);
-            if (fetcher)
-                fetch_u(tid - kSumThreads, kConsumers - kSumThreads, good != 0);
-            else if (lane == 0)
-                s_good = good;
+            fetch_u(tid - kSumThreads, kConsumers - kSumThreads, good != 0);
         } else if (rank == 0 && tid < nsum) {
             const uint32_t red_addr = base + L.red;
             for (int e4 = tid; e4 < tile4; e4 += nsum) {
@@ -599,11 +644,7 @@ decode_w4ec_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_co
             return;
     }
     __syncthreads();
-    if (!kOverlap && p.JB > 0) {
-        if (tid < kConsumers)
-            fetch_u(tid, kConsumers, s_good != 0);
-        __syncthreads();
-    }
+
     if (p.JB > 0 && tid == 0 && atomicAdd(&p.flags[1], 1u) == (unsigned)(p.NC - 1)) {
         // every 64-row cluster has read u: reset for the next forward
         p.flags[1] = 0u;
@@ -853,7 +894,7 @@ void decode_free(DecodeWork &w)
 }
 
 // one partial of u per rank of an EC cluster (at most 8 ranks)
-size_t decode_u_floats(const Packed &pk) { return (size_t)8 * pk.R1p * kUStride; }
+size_t decode_u_floats(const Packed &pk) { return (size_t)(kUFinal + 1) * pk.R1p * kUStride; }
 
 cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, bool ec, const DecodeWork &w,
                           int *status, cudaStream_t st, int num_sms)
@@ -881,7 +922,9 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     p.status = status;
     p.M = M;
     p.N = pk.N;
-    p.JB = use_ec ? pk.R1p / 16 : 0;
+    const int JG = use_ec ? pk.R1p / 16 : 0;   // 16-row groups of G
+    p.JB = JG;
+    p.ES = 1;
     p.NC = (int)(pk.Np / kRows);
     p.Kp = pk.Kp;
     p.r = pk.r;
@@ -917,11 +960,32 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
     const void *fn = nullptr;
     for (int max_cs = 8; max_cs >= 1;) {
         int KS = 0;
-        CS = pick_cluster(pk, num_sms, p.JB, &KS, max_cs);
+        CS = pick_cluster(pk, num_sms, JG, &KS, max_cs);
         if (CS == 0)
             return cudaErrorInvalidValue;
         p.KS = KS;
         p.nch = KS / kChunk;
+        // The EC CTAs stream G (bf16, four times the bytes of a row of codes)
+        // and publish u only when their slice is done, so that the rows wait
+        // for it.  Without a K split (CS = 1) they take 1/ES of K each, ES the
+        // largest (at most 8 partials, no empty slice) that keeps the grid
+        // within two CTAs per SM, so that u is ready before the rows' products
+        // are (MLP up at one token: 15.7 -> 14.9 us per layer with the EC);
+        // with a K split the rows' slices are short already (splitting the EC
+        // CTAs further was measured slower there).
+        const int chunks = (int)(pk.Kp / kChunk);
+        int ES = 1;
+        for (int e = 8 / CS; e > 1 && JG > 0 && CS == 1; --e) {
+            const int per = (chunks + e * CS - 1) / (e * CS);
+            if ((e * CS - 1) * per < chunks && (int64_t)(JG * e + p.NC) * CS <= 2LL * num_sms) {
+                ES = e;
+                break;
+            }
+        }
+        p.ES = ES;
+        p.JB = JG * ES;
+        p.nche = (chunks + ES * CS - 1) / (ES * CS);
+        p.KSe = p.nche * kChunk;
         W = pick_warps(T, p.nch);
         pl = T == 1 ? plan_for<8>(p.nch, p.rp, CS, W)
                     : (T == 2 ? plan_for<16>(p.nch, p.rp, CS, W) : plan_for<32>(p.nch, p.rp, CS, W));

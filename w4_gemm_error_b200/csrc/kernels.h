@@ -83,8 +83,9 @@ int prepass_counters(int64_t max_M);
 // and EC up-projection in the epilogue (when `ec` is set).
 struct DecodeWork {
     void *maps;           // tensor maps of the packed operands (host memory)
-    float *ws_u;          // [8][R1p][32] published partials of the EC down-projection
-    unsigned *flags;      // two counters, zero between calls
+    float *ws_u;          // [9][R1p][32] published partials of the EC down-projection, then their sum
+    unsigned *flags;      // kDecodeFlags counters, zero between calls: [0] groups of G published,
+                          // [1] row clusters done, [2 + g] EC CTAs of group g done
     // codes of the layer that runs next (prefetched into L2 by the decode
     // kernels once their own codes have landed), null for none
     const void *pf;
@@ -96,6 +97,7 @@ struct DecodeWork {
     unsigned *cnt_stream;
 };
 constexpr int kDecodeMaxTokens = 32;   // tokens per launch
+constexpr int kDecodeFlags = 2 + 16;
 bool decode_supported(const Packed &pk, int num_sms);
 cudaError_t decode_prepare(const Packed &pk, DecodeWork &w);
 void decode_free(DecodeWork &w);

@@ -320,7 +320,7 @@ int spear_w4ec_create(spear_w4ec **out, int64_t K, int64_t N, int32_t r, const s
         chk(alloc_zero(&h->pre.counters, (size_t)h->pre.n_counters));
     }
     chk(alloc_zero(&h->dec.ws_u, decode_u_floats(pk)));
-    chk(alloc_zero(&h->dec.flags, (size_t)2));
+    chk(alloc_zero(&h->dec.flags, (size_t)kDecodeFlags));
     chk(alloc_zero(&h->dec.ws_stream, decode_stream_ws_floats(pk)));
     chk(alloc_zero(&h->dec.cnt_stream, (size_t)kDecodeStreamCounters));
     chk(tc_alloc(pk, h->max_M, h->num_sms, h->tc));
