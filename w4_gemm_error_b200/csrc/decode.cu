@@ -975,10 +975,10 @@ cudaError_t launch_decode(const Packed &pk, const void *x, void *y, int64_t M, b
         // CTAs further was measured slower there).
         const int chunks = (int)(pk.Kp / kChunk);
         int ES = 1;
-        for (int e = 8 / CS; e > 1 && JG > 0 && CS == 1; --e) {
-            const int per = (chunks + e * CS - 1) / (e * CS);
-            if ((e * CS - 1) * per < chunks && (int64_t)(JG * e + p.NC) * CS <= 2LL * num_sms) {
-                ES = e;
+        for (int es = 8 / CS; es > 1 && JG > 0 && CS == 1; --es) {
+            const int per = (chunks + es * CS - 1) / (es * CS);
+            if ((es * CS - 1) * per < chunks && (int64_t)(JG * es + p.NC) * CS <= 2LL * num_sms) {
+                ES = es;
                 break;
             }
         }
