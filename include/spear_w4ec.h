@@ -320,6 +320,105 @@ int spear_w4ec_stack_buffer(const spear_w4ec_stack *s, int32_t index, void **ptr
  * left as they are.  NULL is a no-op. */
 int spear_w4ec_stack_destroy(spear_w4ec_stack *s);
 
+/* ---- Row-parallel tensor parallelism: a layer split along K over ranks.
+ *
+ * SPEAR, Abstract: with the EC in a tensor-parallel layer the input-dependent
+ * gate forces a synchronisation between ranks; the pages answer it with a
+ * peer-reduction kernel integrated with the epilogue and a P2P dual write.
+ * This library's reading, for `world` ranks (one per GPU, one process each):
+ * rank p holds the input features [k0_p, k1_p) of the layer, that is
+ *   codes[:, k0_p/8 : k1_p/8] of the exported layout with the per-channel
+ *   s and z of the whole rows, A[k0_p:k1_p, :], w_g[k0_p:k1_p], all of B and b_g,
+ * as an ordinary handle of K = k1_p - k0_p made with spear_w4ec_import (the
+ * scales must be those of the whole row, so do not pack the slice anew), and
+ * receives x_p = x[:, k0_p:k1_p].  Then
+ *   y = sum_p x_p.W^_p^T + g . ((sum_p x_p.A_p) . B),
+ *   g = sigmoid(sum_p x_p.w_g,p + b_g),
+ * where the gate needs the complete [M][r + 1] sum of the partials before the
+ * sigmoid.  One call runs, on each rank's stream:
+ *   partial: waits (bounded) until every rank has finished reading this
+ *            rank's buffers of the previous call, runs the shard's forward
+ *            with the EC off into this rank's partial-output buffer, and
+ *            writes the raw fp32 partials x_p.[w_g,p, A_p] into slot p of
+ *            EVERY rank's exchange buffer (peer stores: the dual write),
+ *            then raises this rank's ready word in every rank's buffer;
+ *   reduce:  waits (bounded) for every rank's ready word, sums the u slots
+ *            in rank order (every rank gets the same u, hence the same gate),
+ *            sums the ranks' partial outputs in rank order (peer loads), adds
+ *            g . (u . B) once and writes the complete y on this rank (an
+ *            all-reduce: every rank holds all of y).  Then it tells every
+ *            rank that it has finished reading their buffers.
+ * Rounding: each rank's partial output is rounded to bf16 once before the
+ * sum, so an element of y is within the single-GPU bound plus about 2^-9 of
+ * the sum over ranks of the partials' magnitudes.
+ * The words that order the ranks count calls on the device, so a sequence of
+ * calls may be captured in a CUDA graph and replayed.  Every rank must make
+ * the same calls with the same M and the same SPEAR_EC_OFF flag.  A wait that
+ * runs out (about a second) sets the timeout bit of the shard handle's
+ * status word (spear_w4ec_sync_status); the group is then out of step and
+ * must be destroyed and created again. */
+typedef struct spear_w4ec_tp spear_w4ec_tp; /* opaque, owned by the library */
+
+/* Largest number of ranks. */
+#define SPEAR_TP_MAX_WORLD 8
+/* Bytes of an exchange buffer's inter-process handle (cudaIpcMemHandle_t). */
+#define SPEAR_TP_IPC_HANDLE_BYTES 64
+
+/* Create rank `rank` (0 <= rank < world <= SPEAR_TP_MAX_WORLD) of a group
+ * over the packed shard handle `shard` (not owned; must outlive the group;
+ * created with max_M at least this max_M) and allocate its exchange buffer
+ * on the shard's device, zeroed: a 256-byte control block, the u slots
+ * [world][max_M][R1] fp32 (R1 = r + 1 rounded up to 16) and the partial
+ * output [max_M][N] bf16.  Every rank of a group must give the same world,
+ * max_M, N and r.  SPEAR_ERR_INVALID for bad arguments, SPEAR_ERR_STATE if
+ * the shard is not packed. */
+int spear_w4ec_tp_create(spear_w4ec_tp **out, spear_w4ec *shard, int32_t rank, int32_t world, int64_t max_M);
+
+/* The exchange buffer of this rank: its device address, its size in bytes
+ * and the byte offsets of the u slots and of the partial output in it (any
+ * of the pointers may be NULL). */
+int spear_w4ec_tp_buffer(const spear_w4ec_tp *t, void **base, size_t *bytes, size_t *u_offset,
+                         size_t *y_offset);
+
+/* The inter-process handle of this rank's exchange buffer, written to
+ * `handle` (SPEAR_TP_IPC_HANDLE_BYTES bytes), to be gathered by every rank. */
+int spear_w4ec_tp_ipc_handle(const spear_w4ec_tp *t, void *handle);
+
+/* Connect the group from the handles of all ranks, `handles` holding world
+ * consecutive SPEAR_TP_IPC_HANDLE_BYTES-byte handles in rank order (this
+ * rank's own entry is not opened; its buffer is used directly).  Opens the
+ * other ranks' buffers with peer access and checks each one's control block
+ * (rank, world, max_M, N, r): SPEAR_ERR_INVALID on a mismatch,
+ * SPEAR_ERR_UNSUPPORTED if a peer's device cannot be reached. */
+int spear_w4ec_tp_connect_ipc(spear_w4ec_tp *t, const void *handles);
+
+/* Connect the group from device addresses that this process can already use
+ * (world entries in rank order, the entry of this rank being its own buffer):
+ * the buffers of other groups' ranks in the same process, on this device or
+ * on a peer device (peer access is enabled here when needed).  The same
+ * checks as spear_w4ec_tp_connect_ipc. */
+int spear_w4ec_tp_connect(spear_w4ec_tp *t, void *const *buffers);
+
+/* The first phase of a call on M tokens (1 <= M <= max_M):
+ *   x   dev bf16 [M][K of the shard] (this rank's columns of the input), 16-byte aligned.
+ * flags: SPEAR_EC_OFF (the plain W4 GEMM on every rank; all ranks must
+ * agree) and SPEAR_FORCE_DECODE / SPEAR_FORCE_TC for the shard's forward.
+ * SPEAR_ERR_STATE before a connect. */
+int spear_w4ec_tp_partial(spear_w4ec_tp *t, const void *x, int64_t M, uint32_t flags, void *stream);
+
+/* The second phase: y dev bf16 [M][N], 16-byte aligned, receives the whole
+ * layer's output.  M and SPEAR_EC_OFF as in the partial phase before it. */
+int spear_w4ec_tp_reduce(spear_w4ec_tp *t, void *y, int64_t M, uint32_t flags, void *stream);
+
+/* Both phases of one call, in order on `stream`. */
+int spear_w4ec_tp_forward(spear_w4ec_tp *t, const void *x, void *y, int64_t M, uint32_t flags,
+                          void *stream);
+
+/* Close the other ranks' buffers and free this rank's (synchronises the
+ * device first).  Every rank must have finished its calls (a barrier of the
+ * caller's) before any rank destroys its group.  NULL is a no-op. */
+int spear_w4ec_tp_destroy(spear_w4ec_tp *t);
+
 /* Human-readable name of a status code (static storage). */
 const char *spear_w4ec_strerror(int status);
 

@@ -99,3 +99,20 @@ def test_table_and_cost_calls_reject_bad_arguments_before_touching_the_device(li
     assert L.spear_w4ec_table_load(None, b"{}") == spear.SPEAR_ERR_INVALID
     assert L.spear_w4ec_cost(None, 1, spear.SPEAR_FORCE_DECODE | spear.SPEAR_FORCE_FUSED, ctypes.byref(us)) \
         == spear.SPEAR_ERR_INVALID
+
+
+def test_tp_calls_reject_bad_arguments_before_touching_the_device(lib):
+    from w4_gemm_error_b200 import spear
+    L = spear.lib()
+    t = ctypes.c_void_p()
+    assert L.spear_w4ec_tp_create(None, None, 0, 1, 1) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_tp_create(ctypes.byref(t), None, 0, 1, 1) == spear.SPEAR_ERR_INVALID   # NULL shard
+    assert t.value is None
+    assert L.spear_w4ec_tp_buffer(None, None, None, None, None) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_tp_ipc_handle(None, None) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_tp_connect_ipc(None, None) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_tp_connect(None, None) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_tp_partial(None, None, 1, 0, None) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_tp_reduce(None, None, 1, 0, None) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_tp_forward(None, None, None, 1, 0, None) == spear.SPEAR_ERR_INVALID
+    assert L.spear_w4ec_tp_destroy(None) == spear.SPEAR_OK

@@ -22,6 +22,7 @@
 #include "async_utils.cuh"
 #include "device_utils.cuh"
 #include "kernels.h"
+#include "tp.h"
 
 namespace spear {
 namespace {
@@ -47,13 +48,21 @@ struct PrepassParams {
     unsigned *counters;   // [tiles] groups summed, then [tiles][kMaxGroups] splits of each group
     unsigned *gcounters;
     unsigned *ready;   // counted (release) once per token tile when its v is written; null for none
+    TpPush push;       // PUSH form: where the raw partials go (tensor-parallel shard)
 };
+
+__device__ __forceinline__ void st_release_sys(unsigned *p, unsigned v)
+{
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 // MINB = 7 caps the registers at 72 per thread, so that a CTA fits on an SM
 // beside a tcgen05 kernel CTA with 64-token tiles (22 warps of 80 registers,
 // about 200 KB of shared memory) at the price of some spills; MINB = 1 is the
-// fast form for a prepass that runs alone.
-template <int MT, int MINB>
+// fast form for a prepass that runs alone.  PUSH: the tensor-parallel form,
+// which writes the raw partial sums of x.G (no bias, no sigmoid) to every
+// rank's slot instead of g and v.
+template <int MT, int MINB, bool PUSH>
 __global__ void __launch_bounds__(128, MINB) prepass_kernel(PrepassParams p)
 {
     pdl_wait();  // x is written by the previous kernel in the stream
@@ -192,6 +201,35 @@ __global__ void __launch_bounds__(128, MINB) prepass_kernel(PrepassParams p)
         __syncthreads();
     }
 
+    if constexpr (PUSH) {
+        // rows of x.G for the tile's tokens, to this rank's slot in every
+        // rank's buffer (peer stores), consecutive threads on consecutive j
+        for (int e = tid; e < kTok * p.R1p; e += 128) {
+            const int tt = e / p.R1p, j = e - tt * p.R1p;
+            const int64_t t = t0 + tt;
+            if (t >= p.M)
+                continue;
+            const float val = red[j * kTok + tt];
+            for (int q = 0; q < p.push.world; ++q)
+                p.push.dst[q][t * p.R1p + j] = val;
+        }
+        __threadfence_system();
+        __syncthreads();
+        if (tid == 0) {
+            const unsigned ntiles = (unsigned)((p.M + kTok - 1) / kTok);
+            if (atomicAdd(p.push.tiles, 1u) == ntiles - 1) {
+                // every tile is written (each writer fenced at system scope
+                // before counting): raise the ready words
+                *p.push.tiles = 0u;
+                __threadfence_system();
+                const unsigned e = *reinterpret_cast<const volatile unsigned *>(p.push.epoch) + 1u;
+                for (int q = 0; q < p.push.world; ++q)
+                    st_release_sys(p.push.ready[q], e);
+            }
+        }
+        return;
+    }
+
     // epilogue: gate and v for the tile's tokens (row 0 of the tile is the logit)
     __shared__ float s_gate[kTok];
     if (tid < kTok) {
@@ -226,23 +264,23 @@ int pick_splits(int64_t M, int64_t Kp, int num_sms)
 }
 
 using PrepassFn = void (*)(PrepassParams);
-template <int MINB>
+template <int MINB, bool PUSH>
 PrepassFn prepass_fn_b(int MT)
 {
     switch (MT) {
-    case 1: return prepass_kernel<1, MINB>;
-    case 2: return prepass_kernel<2, MINB>;
-    case 3: return prepass_kernel<3, MINB>;
-    case 4: return prepass_kernel<4, MINB>;
-    case 5: return prepass_kernel<5, MINB>;
-    case 6: return prepass_kernel<6, MINB>;
-    case 7: return prepass_kernel<7, MINB>;
-    case 8: return prepass_kernel<8, MINB>;
-    case 9: return prepass_kernel<9, MINB>;
+    case 1: return prepass_kernel<1, MINB, PUSH>;
+    case 2: return prepass_kernel<2, MINB, PUSH>;
+    case 3: return prepass_kernel<3, MINB, PUSH>;
+    case 4: return prepass_kernel<4, MINB, PUSH>;
+    case 5: return prepass_kernel<5, MINB, PUSH>;
+    case 6: return prepass_kernel<6, MINB, PUSH>;
+    case 7: return prepass_kernel<7, MINB, PUSH>;
+    case 8: return prepass_kernel<8, MINB, PUSH>;
+    case 9: return prepass_kernel<9, MINB, PUSH>;
     default: return nullptr;
     }
 }
-PrepassFn prepass_fn(int MT, bool slim) { return slim ? prepass_fn_b<7>(MT) : prepass_fn_b<1>(MT); }
+PrepassFn prepass_fn(int MT, bool slim) { return slim ? prepass_fn_b<7, false>(MT) : prepass_fn_b<1, false>(MT); }
 
 }  // namespace
 
@@ -265,12 +303,17 @@ size_t prepass_part_floats(const Packed &pk, int64_t max_M, int num_sms)
 // One counter per token tile for the groups, then kMaxGroups per tile for the splits.
 int prepass_counters(int64_t max_M) { return (int)((max_M + kTok - 1) / kTok) * (1 + kMaxGroups); }
 
-cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
-                           const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready, bool slim)
+namespace {
+
+// push == nullptr: the gate and v (launch_prepass); otherwise the raw
+// partials to the ranks' slots (launch_prepass_partial)
+cudaError_t launch_any(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
+                       const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready, bool slim,
+                       const TpPush *push)
 {
     if (M <= 0 || pk.r == 0)
         return cudaSuccess;
-    PrepassParams p;
+    PrepassParams p = {};
     p.G = pk.G;
     p.x = static_cast<const uint16_t *>(x);
     p.M = M;
@@ -294,9 +337,11 @@ cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v,
     p.counters = w.counters;
     p.gcounters = w.counters + tiles_cap;
     p.ready = ready;
+    if (push)
+        p.push = *push;
     if (tiles > tiles_cap || (p.S > 1 && (size_t)tiles * (p.S + kMaxGroups) * pk.R1p * kTok > w.part_floats))
         return cudaErrorInvalidValue;
-    PrepassFn fn = prepass_fn(pk.R1p / 16, slim);
+    PrepassFn fn = push ? prepass_fn_b<1, true>(pk.R1p / 16) : prepass_fn(pk.R1p / 16, slim);
     if (!fn)
         return cudaErrorInvalidValue;
     const size_t smem = (size_t)4 * pk.R1p * kTok * sizeof(float);
@@ -316,6 +361,22 @@ cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, fn, p);
+}
+
+}  // namespace
+
+cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v, bool tf32, float *g,
+                           const PrepassWork &w, cudaStream_t st, int num_sms, unsigned *ready, bool slim)
+{
+    return launch_any(pk, x, M, v, tf32, g, w, st, num_sms, ready, slim, nullptr);
+}
+
+cudaError_t launch_prepass_partial(const Packed &pk, const void *x, int64_t M, const PrepassWork &w,
+                                   const TpPush &push, cudaStream_t st, int num_sms)
+{
+    if (push.world < 1 || push.world > kTpMaxWorld || !push.epoch || !push.tiles)
+        return cudaErrorInvalidValue;
+    return launch_any(pk, x, M, nullptr, false, nullptr, w, st, num_sms, nullptr, false, &push);
 }
 
 }  // namespace spear

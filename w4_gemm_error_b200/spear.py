@@ -31,13 +31,18 @@ SPEAR_FORCE_DECODE = 8
 SPEAR_FORCE_TC = 16
 SPEAR_STACK_PERSISTENT = 32   # stack forward only: one persistent kernel for the whole stack
 
+SPEAR_TP_MAX_WORLD = 8
+SPEAR_TP_IPC_HANDLE_BYTES = 64
+
 EXPORTED = ("spear_w4ec_create", "spear_w4ec_pack", "spear_w4ec_pack_asym", "spear_w4ec_import",
             "spear_w4ec_forward", "spear_w4ec_forward_host",
             "spear_w4ec_destroy", "spear_w4ec_get_packed", "spear_w4ec_get_gate", "spear_w4ec_sync_status",
             "spear_w4ec_tune", "spear_w4ec_dispatch", "spear_w4ec_gate_noalloc", "spear_w4ec_set_next",
             "spear_w4ec_stack_create", "spear_w4ec_stack_forward", "spear_w4ec_stack_forward_host",
             "spear_w4ec_stack_buffer", "spear_w4ec_stack_destroy", "spear_w4ec_cost", "spear_w4ec_table_save",
-            "spear_w4ec_table_load", "spear_w4ec_strerror")
+            "spear_w4ec_table_load", "spear_w4ec_tp_create", "spear_w4ec_tp_buffer", "spear_w4ec_tp_ipc_handle",
+            "spear_w4ec_tp_connect_ipc", "spear_w4ec_tp_connect", "spear_w4ec_tp_partial", "spear_w4ec_tp_reduce",
+            "spear_w4ec_tp_forward", "spear_w4ec_tp_destroy", "spear_w4ec_strerror")
 
 
 class SpearError(RuntimeError):
@@ -85,6 +90,16 @@ def _load():
         "spear_w4ec_cost": [P, i64, u32, ctypes.POINTER(f32)],
         "spear_w4ec_table_save": [P, ctypes.c_char_p, ctypes.c_size_t, ctypes.POINTER(ctypes.c_size_t)],
         "spear_w4ec_table_load": [P, ctypes.c_char_p],
+        "spear_w4ec_tp_create": [ctypes.POINTER(P), P, i32, i32, i64],
+        "spear_w4ec_tp_buffer": [P, ctypes.POINTER(P), ctypes.POINTER(ctypes.c_size_t),
+                                 ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)],
+        "spear_w4ec_tp_ipc_handle": [P, P],
+        "spear_w4ec_tp_connect_ipc": [P, P],
+        "spear_w4ec_tp_connect": [P, ctypes.POINTER(P)],
+        "spear_w4ec_tp_partial": [P, P, i64, u32, P],
+        "spear_w4ec_tp_reduce": [P, P, i64, u32, P],
+        "spear_w4ec_tp_forward": [P, P, P, i64, u32, P],
+        "spear_w4ec_tp_destroy": [P],
     }
     for name, args in sig.items():
         f = getattr(lib, name)
@@ -242,6 +257,56 @@ def spear_w4ec_stack_buffer(s: int, index: int) -> int:
 
 def spear_w4ec_stack_destroy(s: int):
     _check(_lib.spear_w4ec_stack_destroy(s), "spear_w4ec_stack_destroy")
+
+
+def spear_w4ec_tp_create(shard_h: int, rank: int, world: int, max_M: int) -> int:
+    out = ctypes.c_void_p()
+    _check(_lib.spear_w4ec_tp_create(ctypes.byref(out), shard_h, int(rank), int(world), int(max_M)),
+           "spear_w4ec_tp_create")
+    return out.value
+
+
+def spear_w4ec_tp_buffer(t: int):
+    """(device address, bytes, u-slot offset, partial-output offset) of the exchange buffer."""
+    base, nbytes, uo, yo = ctypes.c_void_p(), ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib.spear_w4ec_tp_buffer(t, ctypes.byref(base), ctypes.byref(nbytes), ctypes.byref(uo),
+                                     ctypes.byref(yo)), "spear_w4ec_tp_buffer")
+    return base.value, nbytes.value, uo.value, yo.value
+
+
+def spear_w4ec_tp_ipc_handle(t: int) -> bytes:
+    buf = ctypes.create_string_buffer(SPEAR_TP_IPC_HANDLE_BYTES)
+    _check(_lib.spear_w4ec_tp_ipc_handle(t, buf), "spear_w4ec_tp_ipc_handle")
+    return buf.raw
+
+
+def spear_w4ec_tp_connect_ipc(t: int, handles):
+    blob = b"".join(handles)
+    if any(len(h) != SPEAR_TP_IPC_HANDLE_BYTES for h in handles):
+        raise ValueError(f"every handle must be {SPEAR_TP_IPC_HANDLE_BYTES} bytes")
+    buf = ctypes.create_string_buffer(blob, len(blob))
+    _check(_lib.spear_w4ec_tp_connect_ipc(t, buf), "spear_w4ec_tp_connect_ipc")
+
+
+def spear_w4ec_tp_connect(t: int, buffers):
+    arr = (ctypes.c_void_p * len(buffers))(*[int(b) for b in buffers])
+    _check(_lib.spear_w4ec_tp_connect(t, arr), "spear_w4ec_tp_connect")
+
+
+def spear_w4ec_tp_partial(t: int, x, M: int, flags: int = 0, stream=None):
+    _check(_lib.spear_w4ec_tp_partial(t, _ptr(x), M, flags, _stream(stream)), "spear_w4ec_tp_partial")
+
+
+def spear_w4ec_tp_reduce(t: int, y, M: int, flags: int = 0, stream=None):
+    _check(_lib.spear_w4ec_tp_reduce(t, _ptr(y), M, flags, _stream(stream)), "spear_w4ec_tp_reduce")
+
+
+def spear_w4ec_tp_forward(t: int, x, y, M: int, flags: int = 0, stream=None):
+    _check(_lib.spear_w4ec_tp_forward(t, _ptr(x), _ptr(y), M, flags, _stream(stream)), "spear_w4ec_tp_forward")
+
+
+def spear_w4ec_tp_destroy(t: int):
+    _check(_lib.spear_w4ec_tp_destroy(t), "spear_w4ec_tp_destroy")
 
 
 class W4ECLinear:
@@ -405,6 +470,128 @@ class W4ECStack:
     def close(self):
         if getattr(self, "h", None):
             spear_w4ec_stack_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def tp_shard_bounds(K: int, world: int):
+    """Input-feature range [k0, k1) of every rank of a layer of K features
+    split along K over ``world`` ranks: contiguous, in rank order, whole words
+    of the exported code layout (multiples of 8), sizes within 8 of each other."""
+    if K % 8 or not 1 <= world <= SPEAR_TP_MAX_WORLD or K // 8 < world:
+        raise ValueError(f"K = {K} must be a multiple of 8 with at least 8 features per rank "
+                         f"(1 <= world = {world} <= {SPEAR_TP_MAX_WORLD})")
+    words = K // 8
+    return [(8 * (words * p // world), 8 * (words * (p + 1) // world)) for p in range(world)]
+
+
+def _contig(a):
+    if isinstance(a, torch.Tensor):
+        return a.contiguous()
+    import numpy as np
+    return np.ascontiguousarray(a)
+
+
+def tp_shard(codes, s, z, A, w_g, k0: int, k1: int):
+    """One rank's part of a packed layer: (codes[:, k0/8:k1/8], s, z, A[k0:k1],
+    w_g[k0:k1]), the codes in the exported layout [N][K/8] and s, z those of
+    the whole rows; B and b_g are whole on every rank.  Slicing only (torch
+    tensors or NumPy arrays); A and w_g may be None for a layer without an EC."""
+    if k0 % 8 or k1 % 8 or not 0 <= k0 < k1 <= codes.shape[1] * 8:
+        raise ValueError(f"bad range [{k0}, {k1})")
+    part = _contig(codes[:, k0 // 8:k1 // 8])
+    return (part, s, z, None if A is None else _contig(A[k0:k1]), None if w_g is None else _contig(w_g[k0:k1]))
+
+
+def tp_gather_handles(handle: bytes, world: int, group=None):
+    """Every rank's exchange-buffer handle, in rank order, gathered over a
+    torch.distributed process group (any backend)."""
+    import torch.distributed as dist
+    out = [None] * world
+    dist.all_gather_object(out, handle, group=group)
+    if len(out) != world or any(not isinstance(h, bytes) or len(h) != SPEAR_TP_IPC_HANDLE_BYTES for h in out):
+        raise ValueError("the group did not return one handle per rank")
+    return out
+
+
+def _device_copy(ptr: int, shape, typestr: str, dtype, device):
+    class _View:   # device memory seen through the CUDA array interface
+        __cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (ptr, False),
+                                    "version": 2, "strides": None}
+
+    torch.cuda.synchronize(device)
+    return torch.as_tensor(_View(), device=device).view(dtype).clone()
+
+
+class W4ECRowParallel:
+    """One rank of a layer split along K over ``world`` ranks
+    (spear_w4ec_tp_*).  ``shard`` is the rank's W4ECLinear: K = k1 - k0 of
+    tp_shard_bounds, made with ``packed=`` from tp_shard of the whole layer's
+    packed codes; it must stay open while this object is used.  Connect once
+    (connect_group over a process group, or connect with buffer addresses of
+    ranks in this process), then call forward (or partial and reduce) on
+    every rank with the same M and flags."""
+
+    def __init__(self, shard: W4ECLinear, rank: int, world: int, max_M: int):
+        self.shard, self.rank, self.world, self.max_M = shard, rank, world, max_M
+        self.K, self.N, self.r = shard.K, shard.N, shard.r
+        self.device = shard.device
+        self.h = spear_w4ec_tp_create(shard.h, rank, world, max_M)
+        self.base, self.nbytes, self.u_off, self.y_off = spear_w4ec_tp_buffer(self.h)
+        self.R1p = (self.r + 1 + 15) // 16 * 16 if self.r else 16
+
+    def ipc_handle(self) -> bytes:
+        return spear_w4ec_tp_ipc_handle(self.h)
+
+    def connect(self, buffers):
+        spear_w4ec_tp_connect(self.h, buffers)
+
+    def connect_ipc(self, handles):
+        spear_w4ec_tp_connect_ipc(self.h, handles)
+
+    def connect_group(self, group=None):
+        self.connect_ipc(tp_gather_handles(self.ipc_handle(), self.world, group))
+
+    def partial(self, x: torch.Tensor, flags: int = 0, stream=None):
+        M = x.shape[0]
+        _dev_bf16(x, (M, self.K), "x")
+        spear_w4ec_tp_partial(self.h, x, M, flags, stream)
+
+    def reduce(self, M: int, flags: int = 0, out: torch.Tensor | None = None, stream=None):
+        y = out if out is not None else torch.empty((M, self.N), dtype=torch.bfloat16, device=self.device)
+        _dev_bf16(y, (M, self.N), "y")
+        spear_w4ec_tp_reduce(self.h, y, M, flags, stream)
+        return y
+
+    def forward(self, x: torch.Tensor, flags: int = 0, out: torch.Tensor | None = None, stream=None):
+        M = x.shape[0]
+        _dev_bf16(x, (M, self.K), "x")
+        y = out if out is not None else torch.empty((M, self.N), dtype=torch.bfloat16, device=x.device)
+        _dev_bf16(y, (M, self.N), "y")
+        spear_w4ec_tp_forward(self.h, x, y, M, flags, stream)
+        return y
+
+    __call__ = forward
+
+    def u_slots(self, M: int) -> torch.Tensor:
+        """A copy of this rank's u slots after a call on M tokens: [world, M, R1p]
+        fp32, slot q holding rank q's x_q.[w_g, A_q] (entries beyond r zero)."""
+        rows = [_device_copy(self.base + self.u_off + 4 * q * self.max_M * self.R1p, (M, self.R1p), "<f4",
+                             torch.float32, self.device) for q in range(self.world)]
+        return torch.stack(rows)
+
+    def partial_output(self, M: int) -> torch.Tensor:
+        """A copy of this rank's partial output x_p.W^_p^T (bf16 [M, N]) after a call."""
+        return _device_copy(self.base + self.y_off, (M, self.N), "<i2", torch.bfloat16, self.device)
+
+    def close(self):
+        if getattr(self, "h", None):
+            spear_w4ec_tp_destroy(self.h)
             self.h = None
 
     def __del__(self):
