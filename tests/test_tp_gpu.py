@@ -103,7 +103,7 @@ class Group:
 
     def check_slots(self, x, what):
         lay, M = self.lay, x.shape[0]
-        slots = [t.u_slots(M).double().numpy() for t in self.tps]
+        slots = [t.u_slots(M).double().cpu().numpy() for t in self.tps]
         for p in range(1, self.world):
             assert np.array_equal(slots[p], slots[0]), f"{what}: rank {p} holds other u slots than rank 0"
         for q, (k0, k1) in enumerate(self.bounds):
