@@ -51,10 +51,6 @@ struct PrepassParams {
     TpPush push;       // PUSH form: where the raw partials go (tensor-parallel shard)
 };
 
-__device__ __forceinline__ void st_release_sys(unsigned *p, unsigned v)
-{
-    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
 
 // MINB = 7 caps the registers at 72 per thread, so that a CTA fits on an SM
 // beside a tcgen05 kernel CTA with 64-token tiles (22 warps of 80 registers,
@@ -213,18 +209,19 @@ __global__ void __launch_bounds__(128, MINB) prepass_kernel(PrepassParams p)
             for (int q = 0; q < p.push.world; ++q)
                 p.push.dst[q][t * p.R1p + j] = val;
         }
-        __threadfence_system();
         __syncthreads();
         if (tid == 0) {
+            // one fence per CTA orders the CTA's stores (before it through
+            // the barrier) ahead of its count
+            tp_fence(p.push.sys);
             const unsigned ntiles = (unsigned)((p.M + kTok - 1) / kTok);
             if (atomicAdd(p.push.tiles, 1u) == ntiles - 1) {
-                // every tile is written (each writer fenced at system scope
-                // before counting): raise the ready words
+                // every tile is written: one fence, then the ready words
                 *p.push.tiles = 0u;
-                __threadfence_system();
+                tp_fence(p.push.sys);
                 const unsigned e = *reinterpret_cast<const volatile unsigned *>(p.push.epoch) + 1u;
                 for (int q = 0; q < p.push.world; ++q)
-                    st_release_sys(p.push.ready[q], e);
+                    tp_store_relaxed(p.push.ready[q], e, p.push.sys);
             }
         }
         return;

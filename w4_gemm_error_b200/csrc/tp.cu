@@ -14,8 +14,8 @@
 //   forward  of the shard with the EC off into rank p's partial output;
 //   push     the prepass's PUSH form: x_p.[w_g,p, A_p] in fp32 to slot p of
 //            every rank's buffer (peer stores), then rank p's ready word in
-//            every rank's buffer raised to the call's count (system-scope
-//            release after the writers' system-scope fences);
+//            every rank's buffer raised to the call's count (one fence per
+//            writing CTA, one before the words, at the group's scope);
 //   reduce   waits for every rank's ready word, sums the u slots in rank
 //            order and the ranks' partial outputs in rank order (peer loads),
 //            adds g . (u . B) once, writes y; its last CTA advances the count
@@ -70,24 +70,22 @@ static_assert(offsetof(TpCtrl, done) == 64 && offsetof(TpCtrl, epoch) == 128 && 
 
 constexpr size_t kCtrlBytes = sizeof(TpCtrl);
 
-__device__ __forceinline__ unsigned ld_acquire_sys(const unsigned *p)
+// Raises this rank's word in every rank's buffer to `e`: one fence at the
+// group's scope (everything this thread has written or observed goes first),
+// then the stores.
+__device__ __forceinline__ void raise_words(unsigned *const *words, int world, unsigned e, int sys)
 {
-    unsigned v;
-    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_sys_word(unsigned *p, unsigned v)
-{
-    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    tp_fence(sys);
+    for (int q = 0; q < world; ++q)
+        tp_store_relaxed(words[q], e, sys);
 }
 
 // Waits (bounded) until the word reaches `target` (counts compared modulo
 // 2^32); false if the wait ran out.
-__device__ __forceinline__ bool wait_count(const unsigned *w, unsigned target)
+__device__ __forceinline__ bool wait_count(const unsigned *w, unsigned target, int sys)
 {
     const long long t0 = clock64();
-    while ((int)(ld_acquire_sys(w) - target) < 0) {
+    while ((int)(tp_load_acquire(w, sys) - target) < 0) {
         if (clock64() - t0 > kWaitBudgetCycles)
             return false;
         __nanosleep(64);
@@ -95,7 +93,7 @@ __device__ __forceinline__ bool wait_count(const unsigned *w, unsigned target)
     return true;
 }
 
-__global__ void __launch_bounds__(32) tp_enter_kernel(const TpCtrl *ctrl, int world, int *status)
+__global__ void __launch_bounds__(32) tp_enter_kernel(const TpCtrl *ctrl, int world, int sys, int *status)
 {
     // the shard's forward may start its weight prefetch now; it waits for
     // this kernel's end before it writes anything
@@ -104,7 +102,7 @@ __global__ void __launch_bounds__(32) tp_enter_kernel(const TpCtrl *ctrl, int wo
     const int q = threadIdx.x;
     if (q < world) {
         const unsigned e = *reinterpret_cast<const volatile unsigned *>(&ctrl->epoch);
-        if (!wait_count(&ctrl->done[q], e))
+        if (!wait_count(&ctrl->done[q], e, sys))
             atomicOr(status, kStatusTimeout);
     }
 }
@@ -113,12 +111,8 @@ __global__ void __launch_bounds__(32) tp_enter_kernel(const TpCtrl *ctrl, int wo
 __global__ void __launch_bounds__(32) tp_signal_kernel(TpPush push)
 {
     pdl_wait();   // the shard's forward has written the partial output
-    if (threadIdx.x == 0) {
-        __threadfence_system();
-        const unsigned e = *reinterpret_cast<const volatile unsigned *>(push.epoch) + 1u;
-        for (int q = 0; q < push.world; ++q)
-            st_release_sys_word(push.ready[q], e);
-    }
+    if (threadIdx.x == 0)
+        raise_words(push.ready, push.world, *reinterpret_cast<const volatile unsigned *>(push.epoch) + 1u, push.sys);
 }
 
 constexpr int kRThreads = 256;   // output channels per CTA (one per thread)
@@ -134,7 +128,7 @@ struct TpReduceParams {
     uint16_t *y;                          // [M][N] bf16
     int *status;
     int64_t M, N;
-    int world, R1p, rp, ec;
+    int world, R1p, rp, ec, sys;
     float b_g;
 };
 
@@ -150,7 +144,7 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
         s_e = *reinterpret_cast<const volatile unsigned *>(&p.ctrl->epoch) + 1u;
     __syncthreads();
     const unsigned e = s_e;
-    if (tid < p.world && !wait_count(&p.ctrl->ready[tid], e))
+    if (tid < p.world && !wait_count(&p.ctrl->ready[tid], e, p.sys))
         atomicOr(p.status, kStatusTimeout);
     __syncthreads();
 
@@ -184,10 +178,12 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
                                      bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
 #pragma unroll
                 for (int i = 0; i < kRTok; ++i) {
-                    const float *ur = us + i * SV + 1 + j;   // u_1 .. u_r follow the logit
+                    if (i < ntok) {
+                        const float *ur = us + i * SV + 1 + j;   // u_1 .. u_r follow the logit
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        corr[i] += ur[q] * bj[q];
+                        for (int q = 0; q < 8; ++q)
+                            corr[i] += ur[q] * bj[q];
+                    }
                 }
             }
 #pragma unroll
@@ -220,9 +216,7 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
             __threadfence();
             p.ctrl->ctas = 0u;
             *reinterpret_cast<volatile unsigned *>(&p.ctrl->epoch) = e;
-            __threadfence_system();
-            for (int q = 0; q < p.world; ++q)
-                st_release_sys_word(p.done[q], e);
+            raise_words(p.done, p.world, e, p.sys);
         }
     }
 }
@@ -256,6 +250,7 @@ struct spear_w4ec_tp {
     void *peer[kTpMaxWorld] = {};
     bool opened[kTpMaxWorld] = {};
     bool connected = false;
+    int sys = 1;    // ordering scope of the group's words: 0 when every buffer is on this device in this process
 };
 
 namespace {
@@ -297,6 +292,7 @@ int run_partial(spear_w4ec_tp *t, const void *x, int64_t M, uint32_t flags, cuda
     TpCtrl *mine = ctrl_of(t->buf);
     TpPush push = {};
     push.world = t->world;
+    push.sys = t->sys;
     push.epoch = &mine->epoch;
     push.tiles = &mine->tiles;
     for (int q = 0; q < t->world; ++q) {
@@ -304,10 +300,10 @@ int run_partial(spear_w4ec_tp *t, const void *x, int64_t M, uint32_t flags, cuda
                       (size_t)t->rank * t->slot_floats;
         push.ready[q] = &ctrl_of(t->peer[q])->ready[t->rank];
     }
-    int world = t->world;
+    int world = t->world, sys = t->sys;
     int *status = h->status;
     const TpCtrl *cm = mine;
-    void *enter_args[] = {&cm, &world, &status};
+    void *enter_args[] = {&cm, &world, &sys, &status};
     cudaError_t e = launch_pdl(reinterpret_cast<const void *>(tp_enter_kernel), dim3(1), dim3(32), 0, st,
                                enter_args);
     if (e != cudaSuccess)
@@ -346,6 +342,7 @@ int run_reduce(spear_w4ec_tp *t, void *y, int64_t M, uint32_t flags, cudaStream_
     p.R1p = t->R1p;
     p.rp = h->pk.rp;
     p.ec = (!(flags & SPEAR_EC_OFF) && t->r > 0) ? 1 : 0;
+    p.sys = t->sys;
     p.b_g = h->pk.b_g;
     const dim3 grid((unsigned)((t->N + kRThreads - 1) / kRThreads), (unsigned)((M + kRTok - 1) / kRTok));
     const size_t smem = (size_t)kRTok * (t->R1p + 16) * sizeof(float);
@@ -484,6 +481,7 @@ int spear_w4ec_tp_connect_ipc(spear_w4ec_tp *t, const void *handles)
         close_peers(t);
         return rc;
     }
+    t->sys = t->world > 1 ? 1 : 0;   // the other ranks are other processes
     t->connected = true;
     return SPEAR_OK;
 }
@@ -498,6 +496,7 @@ int spear_w4ec_tp_connect(spear_w4ec_tp *t, void *const *buffers)
     if (!guard.ok())
         return SPEAR_ERR_CUDA;
     close_peers(t);
+    int sys = 0;
     for (int q = 0; q < t->world; ++q) {
         if (!buffers[q])
             return SPEAR_ERR_INVALID;
@@ -507,6 +506,7 @@ int spear_w4ec_tp_connect(spear_w4ec_tp *t, void *const *buffers)
             return SPEAR_ERR_INVALID;
         }
         if (a.device != t->device) {
+            sys = 1;
             int can = 0;
             if (cudaDeviceCanAccessPeer(&can, t->device, a.device) != cudaSuccess || !can)
                 return SPEAR_ERR_UNSUPPORTED;
@@ -523,6 +523,7 @@ int spear_w4ec_tp_connect(spear_w4ec_tp *t, void *const *buffers)
         close_peers(t);
         return rc;
     }
+    t->sys = sys;
     t->connected = true;
     return SPEAR_OK;
 }
