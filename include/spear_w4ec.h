@@ -386,10 +386,12 @@ int spear_w4ec_tp_ipc_handle(const spear_w4ec_tp *t, void *handle);
 
 /* Connect the group from the handles of all ranks, `handles` holding world
  * consecutive SPEAR_TP_IPC_HANDLE_BYTES-byte handles in rank order (this
- * rank's own entry is not opened; its buffer is used directly).  Opens the
- * other ranks' buffers with peer access and checks each one's control block
- * (rank, world, max_M, N, r): SPEAR_ERR_INVALID on a mismatch,
- * SPEAR_ERR_UNSUPPORTED if a peer's device cannot be reached. */
+ * rank's own entry must be its own handle and is not opened; its buffer is
+ * used directly).  Opens the other ranks' buffers with peer access and
+ * checks each one's control block (rank, world, max_M, N, r):
+ * SPEAR_ERR_INVALID on a mismatch or a handle that cannot be opened,
+ * SPEAR_ERR_UNSUPPORTED if a peer's device cannot be reached, SPEAR_ERR_CUDA
+ * for another failure of the runtime.  On any failure nothing stays open. */
 int spear_w4ec_tp_connect_ipc(spear_w4ec_tp *t, const void *handles);
 
 /* Connect the group from device addresses that this process can already use

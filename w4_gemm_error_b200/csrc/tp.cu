@@ -459,6 +459,17 @@ int spear_w4ec_tp_connect_ipc(spear_w4ec_tp *t, const void *handles)
         return SPEAR_ERR_CUDA;
     close_peers(t);
     const unsigned char *hb = static_cast<const unsigned char *>(handles);
+    // this rank's own entry must be its own handle, and no other entry may be
+    // (a process cannot open its own handle)
+    cudaIpcMemHandle_t own;
+    cudaError_t e = cudaIpcGetMemHandle(&own, t->buf);
+    if (e != cudaSuccess)
+        return status_of(e);
+    for (int q = 0; q < t->world; ++q) {
+        const bool same = std::memcmp(hb + (size_t)q * SPEAR_TP_IPC_HANDLE_BYTES, &own, sizeof(own)) == 0;
+        if (same != (q == t->rank))
+            return SPEAR_ERR_INVALID;
+    }
     for (int q = 0; q < t->world; ++q) {
         if (q == t->rank) {
             t->peer[q] = t->buf;
@@ -467,11 +478,14 @@ int spear_w4ec_tp_connect_ipc(spear_w4ec_tp *t, const void *handles)
         cudaIpcMemHandle_t hd;
         std::memcpy(&hd, hb + (size_t)q * SPEAR_TP_IPC_HANDLE_BYTES, sizeof(hd));
         void *p = nullptr;
-        const cudaError_t e = cudaIpcOpenMemHandle(&p, hd, cudaIpcMemLazyEnablePeerAccess);
+        e = cudaIpcOpenMemHandle(&p, hd, cudaIpcMemLazyEnablePeerAccess);
         if (e != cudaSuccess) {
             cudaGetLastError();
             close_peers(t);
-            return e == cudaErrorPeerAccessUnsupported ? SPEAR_ERR_UNSUPPORTED : SPEAR_ERR_INVALID;
+            if (e == cudaErrorPeerAccessUnsupported)
+                return SPEAR_ERR_UNSUPPORTED;
+            return (e == cudaErrorInvalidValue || e == cudaErrorInvalidResourceHandle) ? SPEAR_ERR_INVALID
+                                                                                       : status_of(e);
         }
         t->peer[q] = p;
         t->opened[q] = true;
