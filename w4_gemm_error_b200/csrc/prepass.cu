@@ -198,6 +198,14 @@ __global__ void __launch_bounds__(128, MINB) prepass_kernel(PrepassParams p)
     }
 
     if constexpr (PUSH) {
+        // the slots this call overwrites are free once every rank has
+        // finished the previous call's reduce
+        if (tid < p.push.world) {
+            const unsigned e = *reinterpret_cast<const volatile unsigned *>(p.push.epoch);
+            if (!tp_wait_count(p.push.done + tid, e, p.push.sys))
+                atomicOr(p.push.status, kStatusTimeout);
+        }
+        __syncthreads();
         // rows of x.G for the tile's tokens, to this rank's slot in every
         // rank's buffer (peer stores), consecutive threads on consecutive j
         for (int e = tid; e < kTok * p.R1p; e += 128) {
@@ -210,20 +218,8 @@ __global__ void __launch_bounds__(128, MINB) prepass_kernel(PrepassParams p)
                 p.push.dst[q][t * p.R1p + j] = val;
         }
         __syncthreads();
-        if (tid == 0) {
-            // one fence per CTA orders the CTA's stores (before it through
-            // the barrier) ahead of its count
-            tp_fence(p.push.sys);
-            const unsigned ntiles = (unsigned)((p.M + kTok - 1) / kTok);
-            if (atomicAdd(p.push.tiles, 1u) == ntiles - 1) {
-                // every tile is written: one fence, then the ready words
-                *p.push.tiles = 0u;
-                tp_fence(p.push.sys);
-                const unsigned e = *reinterpret_cast<const volatile unsigned *>(p.push.epoch) + 1u;
-                for (int q = 0; q < p.push.world; ++q)
-                    tp_store_relaxed(p.push.ready[q], e, p.push.sys);
-            }
-        }
+        if (tid == 0)
+            tp_fence(p.push.sys);   // the CTA's stores (before it through the barrier) reach every rank first
         return;
     }
 
@@ -371,7 +367,7 @@ cudaError_t launch_prepass(const Packed &pk, const void *x, int64_t M, float *v,
 cudaError_t launch_prepass_partial(const Packed &pk, const void *x, int64_t M, const PrepassWork &w,
                                    const TpPush &push, cudaStream_t st, int num_sms)
 {
-    if (push.world < 1 || push.world > kTpMaxWorld || !push.epoch || !push.tiles)
+    if (push.world < 1 || push.world > kTpMaxWorld || !push.epoch || !push.done || !push.status)
         return cudaErrorInvalidValue;
     return launch_any(pk, x, M, nullptr, false, nullptr, w, st, num_sms, nullptr, false, &push);
 }

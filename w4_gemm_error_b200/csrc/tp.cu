@@ -8,14 +8,17 @@
 // before its up-projection); the pages meet it with a peer-reduction kernel
 // and a P2P dual write.  This library's form, per call and rank p:
 //
-//   enter    (one CTA) waits until every rank has finished reading rank p's
-//            buffers of the previous call (their done words reach the count
-//            of completed calls);
-//   forward  of the shard with the EC off into rank p's partial output;
-//   push     the prepass's PUSH form: x_p.[w_g,p, A_p] in fp32 to slot p of
-//            every rank's buffer (peer stores), then rank p's ready word in
-//            every rank's buffer raised to the call's count (one fence per
-//            writing CTA, one before the words, at the group's scope);
+//   push     (with the EC) the prepass's PUSH form: x_p.[w_g,p, A_p] in fp32
+//            to slot p of every rank's buffer (peer stores), its stores held
+//            back (bounded wait) until every rank's done word in rank p's
+//            buffer has reached rank p's count of completed calls: nobody
+//            still reads rank p's buffers of the previous call;
+//   enter    (without the EC; one CTA) the same wait alone;
+//   forward  of the shard with the EC off into rank p's partial output; its
+//            weight copies start while the push runs (programmatic
+//            dependent launch), its writes after the push has ended;
+//   signal   raises rank p's ready word in every rank's buffer to the
+//            call's count (one fence at the group's scope, then the stores);
 //   reduce   waits for every rank's ready word, sums the u slots in rank
 //            order and the ranks' partial outputs in rank order (peer loads),
 //            adds g . (u . B) once, writes y; its last CTA advances the count
@@ -55,9 +58,8 @@ struct TpCtrl {
     unsigned done[kTpMaxWorld];    // rank q has finished reading this buffer for call c: c
     unsigned pad1[8];
     unsigned epoch;                // calls completed by the owner
-    unsigned tiles;                // push: token tiles written in this call
     unsigned ctas;                 // reduce: CTAs finished in this call
-    unsigned pad2[13];
+    unsigned pad2[14];
     // checked by the other ranks when they connect
     uint32_t magic, world, rank, R1p;
     int64_t max_M, N;
@@ -80,19 +82,6 @@ __device__ __forceinline__ void raise_words(unsigned *const *words, int world, u
         tp_store_relaxed(words[q], e, sys);
 }
 
-// Waits (bounded) until the word reaches `target` (counts compared modulo
-// 2^32); false if the wait ran out.
-__device__ __forceinline__ bool wait_count(const unsigned *w, unsigned target, int sys)
-{
-    const long long t0 = clock64();
-    while ((int)(tp_load_acquire(w, sys) - target) < 0) {
-        if (clock64() - t0 > kWaitBudgetCycles)
-            return false;
-        __nanosleep(64);
-    }
-    return true;
-}
-
 __global__ void __launch_bounds__(32) tp_enter_kernel(const TpCtrl *ctrl, int world, int sys, int *status)
 {
     // the shard's forward may start its weight prefetch now; it waits for
@@ -102,12 +91,13 @@ __global__ void __launch_bounds__(32) tp_enter_kernel(const TpCtrl *ctrl, int wo
     const int q = threadIdx.x;
     if (q < world) {
         const unsigned e = *reinterpret_cast<const volatile unsigned *>(&ctrl->epoch);
-        if (!wait_count(&ctrl->done[q], e, sys))
+        if (!tp_wait_count(&ctrl->done[q], e, sys))
             atomicOr(status, kStatusTimeout);
     }
 }
 
-// Raises this rank's ready words when no EC partials are pushed (EC off).
+// Raises this rank's ready words once the shard's forward (and the push or
+// enter kernel before it) has ended.
 __global__ void __launch_bounds__(32) tp_signal_kernel(TpPush push)
 {
     pdl_wait();   // the shard's forward has written the partial output
@@ -144,7 +134,7 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
         s_e = *reinterpret_cast<const volatile unsigned *>(&p.ctrl->epoch) + 1u;
     __syncthreads();
     const unsigned e = s_e;
-    if (tid < p.world && !wait_count(&p.ctrl->ready[tid], e, p.sys))
+    if (tid < p.world && !tp_wait_count(&p.ctrl->ready[tid], e, p.sys))
         atomicOr(p.status, kStatusTimeout);
     __syncthreads();
 
@@ -152,16 +142,17 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
     const int ntok = (int)min((int64_t)kRTok, p.M - t0);
     const int SV = p.R1p + 16;
     if (p.ec) {
-        for (int i = tid; i < kRTok * SV; i += kRThreads) {
+        // the rows of the tokens present (the loops below read no others)
+        for (int i = tid; i < ntok * SV; i += kRThreads) {
             const int tt = i / SV, j = i - tt * SV;
             float u = 0.f;
-            if (tt < ntok && j < p.R1p)
+            if (j < p.R1p)
                 for (int q = 0; q < p.world; ++q)
                     u += __ldcg(p.uslots + q * p.slot_floats + (t0 + tt) * p.R1p + j);
             us[i] = u;
         }
         __syncthreads();
-        if (tid < kRTok)
+        if (tid < ntok)
             s_gate[tid] = 1.0f / (1.0f + expf(-(us[tid * SV] + p.b_g)));
         __syncthreads();
     }
@@ -188,7 +179,8 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
             }
 #pragma unroll
             for (int i = 0; i < kRTok; ++i)
-                corr[i] *= s_gate[i];
+                if (i < ntok)
+                    corr[i] *= s_gate[i];
         }
         float sum[kRTok];
 #pragma unroll
@@ -294,18 +286,23 @@ int run_partial(spear_w4ec_tp *t, const void *x, int64_t M, uint32_t flags, cuda
     push.world = t->world;
     push.sys = t->sys;
     push.epoch = &mine->epoch;
-    push.tiles = &mine->tiles;
+    push.done = mine->done;
+    push.status = h->status;
     for (int q = 0; q < t->world; ++q) {
         push.dst[q] = reinterpret_cast<float *>(static_cast<char *>(t->peer[q]) + t->u_off) +
                       (size_t)t->rank * t->slot_floats;
         push.ready[q] = &ctrl_of(t->peer[q])->ready[t->rank];
     }
-    int world = t->world, sys = t->sys;
-    int *status = h->status;
-    const TpCtrl *cm = mine;
-    void *enter_args[] = {&cm, &world, &sys, &status};
-    cudaError_t e = launch_pdl(reinterpret_cast<const void *>(tp_enter_kernel), dim3(1), dim3(32), 0, st,
-                               enter_args);
+    cudaError_t e;
+    if (ec) {
+        e = launch_prepass_partial(h->pk, x, M, h->pre, push, st, h->num_sms);
+    } else {
+        int world = t->world, sys = t->sys;
+        int *status = h->status;
+        const TpCtrl *cm = mine;
+        void *enter_args[] = {&cm, &world, &sys, &status};
+        e = launch_pdl(reinterpret_cast<const void *>(tp_enter_kernel), dim3(1), dim3(32), 0, st, enter_args);
+    }
     if (e != cudaSuccess)
         return status_of(e);
     void *ypart = static_cast<char *>(t->buf) + t->y_off;
@@ -313,12 +310,8 @@ int run_partial(spear_w4ec_tp *t, const void *x, int64_t M, uint32_t flags, cuda
     const int rc = forward_checked(h, x, ypart, M, path | SPEAR_EC_OFF, st);
     if (rc != SPEAR_OK)
         return rc;
-    if (ec) {
-        e = launch_prepass_partial(h->pk, x, M, h->pre, push, st, h->num_sms);
-    } else {
-        void *sig_args[] = {&push};
-        e = launch_pdl(reinterpret_cast<const void *>(tp_signal_kernel), dim3(1), dim3(32), 0, st, sig_args);
-    }
+    void *sig_args[] = {&push};
+    e = launch_pdl(reinterpret_cast<const void *>(tp_signal_kernel), dim3(1), dim3(32), 0, st, sig_args);
     return e == cudaSuccess ? SPEAR_OK : status_of(e);
 }
 
