@@ -137,7 +137,7 @@ def test_world_of_one_matches_the_oracle(M):
 @pytest.mark.parametrize("world", [2, 3, 4])
 def test_emulated_ranks(world):
     """Ragged shards (K = 1032 over 2, 3, 4 ranks), N not a multiple of 256,
-    rank 33; one, nine and forty tokens (two token blocks of the reduce);
+    rank 33; one, nine and forty tokens (three token blocks of the reduce);
     the EC on and off in alternate calls of the same group."""
     g = Group(1032, 776, 33, world, 40, seed=8100 + world)
     from w4_gemm_error_b200 import spear

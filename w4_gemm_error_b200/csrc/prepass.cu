@@ -317,6 +317,8 @@ cudaError_t launch_any(const Packed &pk, const void *x, int64_t M, float *v, boo
     p.rp = pk.rp;
     p.b_g = pk.b_g;
     p.S = pick_splits(M, pk.Kp, num_sms);
+    if (push)
+        p.S = std::min(p.S, kGroup);   // one level of sums: the push form is on the critical path
     const int nkb = (int)(pk.Kp / 64);
     p.bps = (nkb + p.S - 1) / p.S;
     p.S = (nkb + p.bps - 1) / p.bps;  // drop empty splits

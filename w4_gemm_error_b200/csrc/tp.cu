@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(32) tp_signal_kernel(TpPush push)
 }
 
 constexpr int kRThreads = 256;   // output channels per CTA (one per thread)
-constexpr int kRTok = 32;        // tokens per CTA
+constexpr int kRTok = 16;        // tokens per CTA
 
 struct TpReduceParams {
     const uint16_t *ypart[kTpMaxWorld];   // every rank's partial output [M][N]
@@ -127,9 +127,15 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
     extern __shared__ float us[];   // [kRTok][R1p + 16]: the summed u rows (zero beyond R1p)
     __shared__ float s_gate[kRTok];
     __shared__ unsigned s_e;
-    pdl_launch_dependents();
-    pdl_wait();   // this rank's push (or signal) kernel and the forward before it are complete
     const int tid = threadIdx.x;
+    const int64_t n = (int64_t)blockIdx.x * kRThreads + tid;
+    // the first 32 entries of row n of B^T (weights: no wait needed)
+    uint4 b0[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        b0[c] = (p.ec && n < p.N && 8 * c < p.rp) ? ld_nc(p.Bt + n * p.rp + 8 * c) : make_uint4(0, 0, 0, 0);
+    pdl_launch_dependents();
+    pdl_wait();   // this rank's signal kernel and the kernels before it are complete
     if (tid == 0)
         s_e = *reinterpret_cast<const volatile unsigned *>(&p.ctrl->epoch) + 1u;
     __syncthreads();
@@ -156,24 +162,42 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
             s_gate[tid] = 1.0f / (1.0f + expf(-(us[tid * SV] + p.b_g)));
         __syncthreads();
     }
-    const int64_t n = (int64_t)blockIdx.x * kRThreads + tid;
     if (n < p.N) {
+        // rank 0's partial output first, so that its loads are in flight
+        // during the EC; the other ranks' follow in rank order
+        float sum[kRTok];
+        {
+            const unsigned short *src = reinterpret_cast<const unsigned short *>(p.ypart[0]) + t0 * p.N + n;
+#pragma unroll
+            for (int i = 0; i < kRTok; ++i)
+                sum[i] = i < ntok ? __uint_as_float((uint32_t)__ldcg(src + (int64_t)i * p.N) << 16) : 0.f;
+        }
         float corr[kRTok];
 #pragma unroll
         for (int i = 0; i < kRTok; ++i)
             corr[i] = 0.f;
         if (p.ec) {
-            for (int j = 0; j < p.rp; j += 8) {
-                const uint4 bv = ld_nc(p.Bt + n * p.rp + j);
-                const float bj[8] = {bf16_lo(bv.x), bf16_hi(bv.x), bf16_lo(bv.y), bf16_hi(bv.y),
-                                     bf16_lo(bv.z), bf16_hi(bv.z), bf16_lo(bv.w), bf16_hi(bv.w)};
+            // 32 entries of the row per round, their four loads in flight together
+            for (int j0 = 0; j0 < p.rp; j0 += 32) {
+                uint4 bv[4];
 #pragma unroll
-                for (int i = 0; i < kRTok; ++i) {
-                    if (i < ntok) {
-                        const float *ur = us + i * SV + 1 + j;   // u_1 .. u_r follow the logit
+                for (int c = 0; c < 4; ++c)
+                    bv[c] = j0 == 0 ? b0[c]
+                                    : (j0 + 8 * c < p.rp ? ld_nc(p.Bt + n * p.rp + j0 + 8 * c) : make_uint4(0, 0, 0, 0));
 #pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            corr[i] += ur[q] * bj[q];
+                for (int c = 0; c < 4; ++c) {
+                    if (j0 + 8 * c >= p.rp)
+                        break;
+                    const float bj[8] = {bf16_lo(bv[c].x), bf16_hi(bv[c].x), bf16_lo(bv[c].y), bf16_hi(bv[c].y),
+                                         bf16_lo(bv[c].z), bf16_hi(bv[c].z), bf16_lo(bv[c].w), bf16_hi(bv[c].w)};
+#pragma unroll
+                    for (int i = 0; i < kRTok; ++i) {
+                        if (i < ntok) {
+                            const float *ur = us + i * SV + 1 + j0 + 8 * c;   // u_1 .. u_r follow the logit
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                corr[i] += ur[q] * bj[q];
+                        }
                     }
                 }
             }
@@ -182,11 +206,7 @@ __global__ void __launch_bounds__(kRThreads) tp_reduce_kernel(TpReduceParams p)
                 if (i < ntok)
                     corr[i] *= s_gate[i];
         }
-        float sum[kRTok];
-#pragma unroll
-        for (int i = 0; i < kRTok; ++i)
-            sum[i] = 0.f;
-        for (int q = 0; q < p.world; ++q) {
+        for (int q = 1; q < p.world; ++q) {
             const unsigned short *src = reinterpret_cast<const unsigned short *>(p.ypart[q]) + t0 * p.N + n;
 #pragma unroll
             for (int i = 0; i < kRTok; ++i)

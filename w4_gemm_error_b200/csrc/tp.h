@@ -34,8 +34,8 @@ struct TpPush {
 #include "async_utils.cuh"
 
 // The ordering operations of the group at its scope: the system when some
-// rank is on another GPU, else the GPU (a system-scope fence costs several
-// microseconds on B200).
+// rank is on another GPU, else the GPU (on B200 a system-scope fence takes
+// about 1.5 us longer than a GPU-scope one).
 __device__ __forceinline__ void tp_fence(int sys)
 {
     if (sys)
