@@ -1,7 +1,8 @@
-"""Host side of the row-parallel (split-K) layer on CPU: the shard bounds, the
-shard slicing of the binding, the handle exchange over a process group, and
-the decomposition the library's kernels implement, checked with two and
-three gloo ranks against the fp64 oracle of the whole layer.
+"""Host side of the tensor-parallel layer on CPU: the shard bounds, the shard
+slicing of the binding (split along K, and along N for column parallelism),
+the handle exchange over a process group, and the row-parallel
+decomposition the library's kernels implement, checked with two and three
+gloo ranks against the fp64 oracle of the whole layer.
 
 The decomposition (SPEAR, Abstract: the input-dependent gate is what makes
 tensor-parallel ranks synchronise): with rank p holding the input features
@@ -72,6 +73,30 @@ def test_shard_slices_the_exported_layout():
 
 def _f64(t):
     return t.float().double().numpy()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_column_shards_give_the_columns_of_the_whole_layer(world):
+    """Split along N, each rank's oracle forward is exactly its columns of
+    the whole layer's (same u and gate on every rank, same sums per
+    element), with the EC on and off."""
+    import oracle
+    from w4_gemm_error_b200.inputs import make_layer, make_x
+    from w4_gemm_error_b200.spear import tp_column_shard, tp_shard_bounds
+    M, K, N, r = 3, 264, 200, 12
+    lay = make_layer(K, N, r, seed=21)
+    x = make_x(M, K, seed=21)
+    codes, s, z = oracle.pack(lay.W)
+    for ec_on in (True, False):
+        ref = oracle.forward(x, codes, s, z, lay.A, lay.B, lay.wg, lay.b_g, ec_on=ec_on)
+        cols = []
+        for n0, n1 in tp_shard_bounds(N, world):
+            c_p, s_p, z_p, B_p = tp_column_shard(codes, s, z, lay.B, n0, n1)
+            assert c_p.shape == (n1 - n0, K // 8) and B_p.shape == (r, n1 - n0)
+            cols.append(oracle.forward(x, c_p, s_p, z_p, lay.A, B_p, lay.wg, lay.b_g, ec_on=ec_on))
+        assert np.array_equal(np.concatenate(cols, axis=1), ref)
+    with pytest.raises(ValueError):
+        tp_column_shard(codes, s, z, lay.B, 4, 16)
 
 
 def _rank_main(rank, world, port, q, case):

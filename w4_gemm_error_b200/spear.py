@@ -508,6 +508,19 @@ def tp_shard(codes, s, z, A, w_g, k0: int, k1: int):
     return (part, s, z, None if A is None else _contig(A[k0:k1]), None if w_g is None else _contig(w_g[k0:k1]))
 
 
+def tp_column_shard(codes, s, z, B, n0: int, n1: int):
+    """One rank's part of a layer split along N (column parallelism: no
+    exchange, each rank an ordinary handle of its output channels):
+    (codes[n0:n1], s[n0:n1], z[n0:n1], B[:, n0:n1]); A, w_g and b_g are
+    whole on every rank, so every rank forms the same u and gate and its
+    forward gives y[:, n0:n1].  Slicing only; tp_shard_bounds(N, world)
+    gives ranges of whole 8-row groups (a handle's N is a multiple of 8)."""
+    if n0 % 8 or n1 % 8 or not 0 <= n0 < n1 <= codes.shape[0]:
+        raise ValueError(f"bad range [{n0}, {n1})")
+    return (_contig(codes[n0:n1]), _contig(s[n0:n1]), _contig(z[n0:n1]),
+            None if B is None else _contig(B[:, n0:n1]))
+
+
 def tp_gather_handles(handle: bytes, world: int, group=None):
     """Every rank's exchange-buffer handle, in rank order, gathered over a
     torch.distributed process group (any backend)."""
