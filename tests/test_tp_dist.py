@@ -128,6 +128,11 @@ def _rank_main(rank, world, port, q, case):
         dist.all_gather_object(parts, (rank, y_p, u_p))
         handles = tp_gather_handles(bytes([rank]) * 64, world)
         assert [h[0] for h in handles] == list(range(world))
+        try:   # one rank with a short handle: every rank refuses the gathered list
+            tp_gather_handles(b"x" * (63 if rank == world - 1 else 64), world)
+            raise AssertionError("a short handle was accepted")
+        except ValueError:
+            pass
         assert [p[0] for p in parts] == list(range(world))
         y = sum(p[1] for p in parts)
         if r:
