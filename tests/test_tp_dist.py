@@ -169,3 +169,46 @@ def test_ranks_reassemble_the_whole_layer(world, case):
     assert out[0][2][0] == 0 and out[-1][2][1] == case[1]
     for rank, err, _ in out:
         assert err < 1e-12, (rank, err)
+
+
+def _connect_rank(rank, world, port, q):
+    """connect_group of the binding over gloo, with the two library calls it
+    makes replaced by recorders (no GPU here)."""
+    import datetime
+    import sys
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+        from w4_gemm_error_b200 import spear
+        seen = {}
+        spear.spear_w4ec_tp_ipc_handle = lambda h: bytes([10 + rank]) * spear.SPEAR_TP_IPC_HANDLE_BYTES
+        spear.spear_w4ec_tp_connect_ipc = lambda h, handles: seen.setdefault("handles", list(handles))
+        tp = object.__new__(spear.W4ECRowParallel)   # no device: only the host logic runs
+        tp.h, tp.rank, tp.world = 1234, rank, world
+        tp.connect_group()
+        tp.h = None                                    # nothing to destroy
+        q.put((rank, [h[0] for h in seen["handles"]]))
+    except BaseException as exc:
+        q.put((rank, repr(exc)))
+        raise
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_connect_group_hands_every_rank_the_handles_in_rank_order(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_connect_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    want = [10 + r for r in range(world)]
+    assert out == [(r, want) for r in range(world)]
